@@ -1,0 +1,457 @@
+"""Benchmark of the CSA / HCA decode hot path on B200.
+
+Default workload: one CSA decode step at 128K context, batch 32 (64 query
+heads x 512, FP8 entries with a scale per 64, MXFP4 indexer 64 x 128, top-k
+512, window 128 bf16, sink).  A step is one csa_decode call: indexer ->
+top-k -> sparse attention (+ split-K combine) over the whole batch.  The HCA
+decode step at 1M context, batch 8, is timed in the same run and reported
+under "hca_decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Timing: W untimed steps, then K steps, each bracketed by CUDA events on the
+launching stream with an L2 flush (a 256 MB write) between steps outside the
+events; barrier + synchronize on both sides; max over ranks.  Multi-GPU runs
+are independent replicas (weak scaling): each rank decodes its own batch.
+The reference arm (--impl reference) is the CPU oracle on a bounded sample of
+the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA/HCA attn decode tok/s @128K–1M; HBM GB/s & tensor-core % of B200 peak"
+WORKLOAD = "csa_decode_128k_b32"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------ algorithmic bytes
+def csa_decode_bytes(w):
+    """Bytes one CSA decode step must move (per batch): indexer keys of every
+    visible block (E2M1 + E8M0), the indexer query, the selected FP8 entries
+    (codes + scales), the bf16 window, q, and the bf16 output."""
+    nb = w.n_ctx // w.m
+    ne = (w.n_ctx - w.W) // w.m
+    key = w.dI // 2 + w.dI // 32
+    ent = w.d + 4 * (w.d // 64)
+    per_seq = ne * key + w.HI * key + w.HI * 4 + w.k * ent + w.W * w.d * 2 + 2 * w.H * w.d * 2
+    return {"indexer": w.batch * (ne * key + w.HI * key + w.HI * 4 + ne * 4),
+            "attention": w.batch * (w.k * ent + w.W * w.d * 2 + 2 * w.H * w.d * 2),
+            "step": w.batch * per_seq, "n_blocks": nb}
+
+
+def hca_decode_bytes(w):
+    ne = (w.n_ctx - w.W) // w.m
+    ent = w.d + 4 * (w.d // 64)
+    return w.batch * (ne * ent + w.W * w.d * 2 + 2 * w.H * w.d * 2)
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+def setup_csa_decode(w, dev):
+    import torch
+
+    import compressed_sparse_attention_13_b200 as K
+    from synth.workloads import draw_torch
+
+    B, H, d, HI, dI, m, W, k = w.batch, w.H, w.d, w.HI, w.dI, w.m, w.W, w.k
+    nb = w.n_ctx // m
+    p = K.params(m, W, k, H, d, HI, dI, w.scale, K.BF16, K.FP8_S64, K.MXFP4)
+
+    def quant(name, fmt):
+        v = draw_torch(w, name, device=dev)
+        v = v.reshape(-1, v.shape[-1])
+        st = K.empty_stored(fmt, v.shape[0], v.shape[1], device=dev)
+        K.csa_quantize(v, st)
+        torch.cuda.synchronize()
+        return st
+
+    S = {"p": p, "nb": nb}
+    S["kv"] = quant("kv", K.FP8_S64)
+    S["kI"] = quant("kI", K.MXFP4)
+    S["qI"] = quant("qI", K.MXFP4)
+    S["q"] = draw_torch(w, "q", device=dev)
+    S["w"] = draw_torch(w, "w", device=dev)
+    S["window"] = draw_torch(w, "window", device=dev)
+    S["sinks"] = draw_torch(w, "sinks", device=dev)
+    q_pos = torch.full((B,), w.n_ctx, dtype=torch.int64, device=dev)
+    S["q_pos"], S["raw_pos0"] = q_pos, q_pos - W + 1
+    S["out"] = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
+    S["sel"] = torch.empty(B, k, dtype=torch.int32, device=dev)
+    S["ws"] = torch.empty(K.csa_workspace_size(p, K.OP_DECODE, B, 1, nb), dtype=torch.uint8, device=dev)
+    return S
+
+
+def csa_decode_call(w, S, stream=None):
+    import compressed_sparse_attention_13_b200 as K
+    K.csa_decode(S["p"], w.batch, S["q"], S["qI"], S["w"], S["kv"], S["kI"], S["nb"], S["window"],
+                 w.W, S["raw_pos0"], S["q_pos"], S["sinks"], S["out"], S["sel"], S["ws"], stream)
+
+
+def time_steps(fn, steps, warmup, flush, stream):
+    """Per-step CUDA-event times (ms) with an L2 flush before every step."""
+    import torch
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "compressed_sparse_attention_13_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, src_hash):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on
+    the current source of that kernel."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(kernel)
+        if rec and rec.get("source_sha") == src_hash:
+            return rec["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import compressed_sparse_attention_13_b200 as K
+    from synth.workloads import WORKLOADS
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    K.lib()
+    hbm_peak, bf16_peak, peak_kind = peaks()
+
+    w = WORKLOADS[WORKLOAD]
+    S = setup_csa_decode(w, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    step = lambda: csa_decode_call(w, S)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # warm-up + timed steps (the clocks sampler runs across the timed region)
+    barrier()
+    with ClockSampler(local) as clk:
+        times = time_steps(step, args.steps, args.warmup, flush, stream)
+        barrier()
+    t_ms = sum(times)
+    if world > 1:
+        tt = torch.tensor([t_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_ms = float(tt.item())
+    assert K.csa_device_status(reset=True) == 0
+    tokens = w.batch * args.steps * world
+    value = tokens / (t_ms / 1e3)
+
+    # per-kernel times of the decode step (same launch configuration)
+    nb = S["nb"]
+    scores = S["ws"].view(torch.float32)[: w.batch * nb].view(w.batch, nb)
+    kfn = {
+        "indexer_score": lambda: K.indexer_score(S["p"], w.batch, 1, S["qI"], S["w"], S["kI"], nb,
+                                                 S["q_pos"], scores, nb),
+        "topk_select": lambda: K.topk_select(S["p"], w.batch, 1, scores, nb, nb, S["q_pos"], S["sel"]),
+    }
+    ws_attn = torch.empty(K.csa_workspace_size(S["p"], K.OP_SPARSE_ATTN, w.batch, 1, 0),
+                          dtype=torch.uint8, device=dev)
+    kfn["sparse_mqa_attn"] = lambda: K.sparse_mqa_attn(
+        S["p"], w.batch, 1, S["q"], S["kv"], nb, S["sel"], S["window"], w.W, S["raw_pos0"],
+        S["q_pos"], S["sinks"], S["out"], ws_attn)
+    kt = {name: statistics.mean(time_steps(fn, max(20, args.steps // 5), 3, flush, stream))
+          for name, fn in kfn.items()}
+    by = csa_decode_bytes(w)
+    idx_gbs = by["indexer"] / (kt["indexer_score"] / 1e3) / 1e9
+    src = kernel_source_hash(["k_indexer_simt.cu", "common.cuh"])
+
+    # end to end: host inputs (pinned) -> device, step, output -> host
+    host = {n: S[n].detach().cpu().pin_memory() for n in ("q", "w", "window", "q_pos", "raw_pos0")}
+    host["qI"] = S["qI"].data.cpu().pin_memory()
+    host["qI_s"] = S["qI"].scales.cpu().pin_memory()
+    out_h = torch.empty(S["out"].shape, dtype=S["out"].dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        for n in ("q", "w", "window", "q_pos", "raw_pos0"):
+            S[n].copy_(host[n], non_blocking=True)
+        S["qI"].data.copy_(host["qI"], non_blocking=True)
+        S["qI"].scales.copy_(host["qI_s"], non_blocking=True)
+        step()
+        out_h.copy_(S["out"], non_blocking=True)
+
+    e2e_steps = max(10, args.steps // 5)
+    e2e_times = time_steps(e2e_step, e2e_steps, 3, flush, stream)
+    e2e_value = w.batch * e2e_steps / (sum(e2e_times) / 1e3)
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp32 (SIMT) on fp8/mxfp4/bf16 inputs", "data": "synthetic (seeded N(0,1))",
+        "config": {"workload": WORKLOAD, "batch": w.batch, "context": w.n_ctx, "heads": w.H,
+                   "head_dim": w.d, "idx_heads": w.HI, "idx_dim": w.dI, "m": w.m, "top_k": w.k,
+                   "window": w.W, "kv": "fp8_e4m3_scale64", "indexer": "mxfp4",
+                   "parallelism": f"replicas x{world}", "l2": "flushed (256 MB write) between steps"},
+        "roofline": {"kernel": "indexer_score", "bound": "hbm", "achieved": round(idx_gbs, 1),
+                     "peak": hbm_peak, "unit": "GB/s", "frac": round(idx_gbs / hbm_peak, 4),
+                     "traffic": recorded_traffic("indexer_score", src),
+                     "algorithmic_bytes": by["indexer"], "peak_source": peak_kind},
+        "kernels_us": {n: round(v * 1e3, 2) for n, v in kt.items()},
+        "step_bytes": by["step"],
+        "step_gbs": round(by["step"] / (t_ms / args.steps / 1e3) / 1e9, 1),
+        "e2e": {"value": round(e2e_value, 1), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and rank == 0 and not args.no_extra:
+        result["hca_decode"] = bench_hca(args, dev, flush, stream, hbm_peak)
+        del S
+        torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def bench_hca(args, dev, flush, stream, hbm_peak):
+    """HCA decode at 1M context, batch 8: pool the context (m' = 128) into FP8
+    entries once, then time hca_attn steps."""
+    import torch
+
+    import compressed_sparse_attention_13_b200 as K
+    from synth.workloads import WORKLOADS, draw_torch
+
+    w = WORKLOADS["hca_decode_1m_b8"]
+    B, N, H, d, m, W = w.batch, w.n_ctx, w.H, w.d, w.m, w.W
+    nb = N // m
+    p = K.params(m, W, 1, H, d, 1, 32, w.scale, K.BF16, K.FP8_S64, K.MXFP4)
+    kv = K.empty_stored(K.FP8_S64, B * nb, d, device=dev)
+    bias = draw_torch(w, "bias", device=dev)
+    x = draw_torch(w, "x", device=dev)
+    z = draw_torch(w, "z", device=dev)
+    comp = lambda: K.csa_compress(p, d, x, z, bias, B * N, kv)
+    t_comp = statistics.mean(time_steps(comp, 5, 1, flush, stream))
+    comp_bytes = 2 * B * N * d * 2 + B * nb * (d + 4 * d // 64)
+    win = torch.cat([x[:, N - W + 1:], draw_torch(w, "x_new", device=dev)[:, None]], 1).contiguous()
+    del x, z
+    torch.cuda.empty_cache()
+    q, sinks = draw_torch(w, "q", device=dev), draw_torch(w, "sinks", device=dev)
+    q_pos = torch.full((B,), N, dtype=torch.int64, device=dev)
+    out = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(K.csa_workspace_size(p, K.OP_HCA_ATTN, B, 1, nb), dtype=torch.uint8, device=dev)
+    fn = lambda: K.hca_attn(p, B, 1, q, kv, nb, win, W, q_pos - W + 1, q_pos, sinks, out, ws)
+    times = time_steps(fn, args.steps, args.warmup, flush, stream)
+    t = statistics.mean(times)
+    by = hca_decode_bytes(w)
+    gbs = by / (t / 1e3) / 1e9
+    return {"workload": "hca_decode_1m_b8", "value": round(B / (t / 1e3), 1), "unit": "tok/s",
+            "ms_per_step": round(t, 5), "step_bytes": by,
+            "roofline": {"kernel": "hca_attn", "bound": "hbm", "achieved": round(gbs, 1),
+                         "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4)},
+            "compress": {"workload": "pool 8 x 1M bf16 tokens at m'=128 -> FP8",
+                         "ms": round(t_comp, 3), "bytes": comp_bytes,
+                         "achieved_gbs": round(comp_bytes / (t_comp / 1e3) / 1e9, 1)}}
+
+
+# ------------------------------------------------------------- CPU oracle
+def _oracle_sample(w, seqs):
+    """Host inputs for the sampled sequences, quantised by the oracle."""
+    import oracle
+    from synth.workloads import draw_np
+    sinks = draw_np(w, "sinks")
+    rows = []
+    for b in seqs:
+        v = {n: draw_np(w, n, b) for n in ("q", "qI", "w", "kv", "kI", "window")}
+        rows.append(dict(q=oracle.Stored(oracle.BF16, v["q"]), kv=oracle.quantize_fp8_s64(v["kv"]),
+                         qI=oracle.quantize_mxfp4(v["qI"]), w=v["w"][None], kI=oracle.quantize_mxfp4(v["kI"]),
+                         win=oracle.Stored(oracle.BF16, v["window"])))
+    return rows, sinks
+
+
+def _oracle_step(w, rows, sinks, threads):
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    t = w.n_ctx
+
+    def one(r):
+        return oracle.csa(r["q"], r["kv"], r["qI"], r["w"], r["kI"], r["win"], t - w.W + 1, sinks,
+                          [t], w.H, w.HI, w.m, w.W, w.k, w.scale, 1)
+
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(one, rows))
+
+
+def cpu_baseline(w, seconds):
+    """The oracle, as it stands, on all host cores: one sequence per thread,
+    repeated until about `seconds` of CPU work."""
+    import oracle
+    oracle.build()
+    cores = os.cpu_count() or 1
+    n = min(cores, 8)
+    rows, sinks = _oracle_sample(w, list(range(n)))
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        _oracle_step(w, rows, sinks, n)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el * n >= seconds or el > seconds:
+            break
+    return {"value": round(reps * n / el, 3), "unit": "tok/s", "cores": n, "kind": "oracle",
+            "sample": f"{reps} x {n} sequences of the {w.batch}-sequence batch (one thread each), "
+                      f"{el:.1f} s wall"}
+
+
+def run_reference(args):
+    """The CPU oracle timed as the reference arm on the same workload and metric."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from synth.workloads import WORKLOADS
+    oracle.build()
+    w = WORKLOADS[WORKLOAD]
+    cores = os.cpu_count() or 1
+    n = min(cores, 16)
+    rows, sinks = _oracle_sample(w, list(range(n)))
+    for _ in range(args.warmup):
+        _oracle_step(w, rows, sinks, n)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(w, rows, sinks, n)
+    el = time.perf_counter() - t0
+    value = n * args.steps / el
+    res = {"metric": METRIC, "value": round(value, 3), "unit": "tok/s", "impl": "reference",
+           "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded N(0,1))",
+           "config": {"workload": WORKLOAD, "batch": w.batch, "context": w.n_ctx, "heads": w.H,
+                      "head_dim": w.d, "top_k": w.k, "window": w.W},
+           "cpu_baseline": {"value": round(value, 3), "unit": "tok/s", "cores": n, "kind": "oracle",
+                            "sample": f"each step: {n} of the {w.batch} sequences, one thread each"},
+           "e2e": {"value": round(value, 3), "unit": "tok/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the HCA decode leg")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,347 @@
+// C-ABI entry points (declared in include/csa.h): argument checks on the
+// host, workspace layout, and the choice of kernel for each format.
+#include <stdio.h>
+
+#include "kernels.h"
+
+namespace csa {
+
+__device__ unsigned int g_status = 0;
+
+static bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+static bool act_ok(int f) { return f == CSA_F32 || f == CSA_BF16; }
+static bool kv_ok(int f) { return f == CSA_F32 || f == CSA_BF16 || f == CSA_FP8_S64; }
+static bool idx_ok(int f) { return f == CSA_F32 || f == CSA_BF16 || f == CSA_MXFP4; }
+
+static int check_params(const csa_params* p, bool need_idx, bool need_attn) {
+    if (!p) return CSA_ERR_ARG;
+    if (p->m <= 0 || p->window < 0) return CSA_ERR_ARG;
+    if (need_attn) {
+        if (p->n_heads <= 0 || p->head_dim <= 0 || (p->head_dim % 64) != 0) return CSA_ERR_ARG;
+        if (!act_ok(p->act_fmt) || !kv_ok(p->kv_fmt)) return CSA_ERR_ARG;
+        if (!(p->scale == p->scale)) return CSA_ERR_ARG;
+    }
+    if (need_idx) {
+        if (p->idx_heads <= 0 || p->idx_dim <= 0 || (p->idx_dim % 32) != 0) return CSA_ERR_ARG;
+        if (!idx_ok(p->idx_fmt) || p->top_k <= 0) return CSA_ERR_ARG;
+    }
+    return CSA_OK;
+}
+
+static int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return CSA_OK;
+    if (e == cudaErrorInvalidValue) return CSA_ERR_UNSUPPORTED;
+    return CSA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ attention
+static int choose_splits(int64_t rows, int64_t items_per_row) {
+    // Enough CTAs to cover every SM about twice, with at least 64 items per split.
+    if (rows >= 2 * kNumSMs) return 1;
+    int64_t s = ceil_div(2 * kNumSMs, rows);
+    s = std::min<int64_t>(s, ceil_div(items_per_row, 64));
+    return int(std::max<int64_t>(1, std::min<int64_t>(s, 64)));
+}
+
+struct AttnPlan {
+    int n_splits;
+    size_t part_o_bytes, part_ml_bytes;
+    size_t bytes() const { return n_splits > 1 ? part_o_bytes + part_ml_bytes : 0; }
+};
+
+static AttnPlan plan_attn(const csa_params* p, int64_t rows, int64_t items_per_row) {
+    AttnPlan a;
+    a.n_splits = choose_splits(rows, items_per_row);
+    const int64_t items = rows * a.n_splits;
+    a.part_o_bytes = size_t(items) * p->n_heads * p->head_dim * sizeof(float);
+    a.part_ml_bytes = size_t(items) * p->n_heads * sizeof(float2);
+    a.part_o_bytes = (a.part_o_bytes + 255) & ~size_t(255);
+    return a;
+}
+
+static int run_attn(const csa_params* p, int batch, int n_q, const void* q, const void* kv,
+                    const void* kv_s, int64_t max_entries, const int32_t* idx, const void* raw,
+                    int64_t n_raw, const int64_t* raw_pos0, const int64_t* q_pos,
+                    const float* sinks, void* out, void* ws, size_t ws_bytes, int64_t items_per_row,
+                    cudaStream_t s) {
+    const int64_t rows = int64_t(batch) * n_q;
+    if (!attn_simt_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim))
+        return CSA_ERR_UNSUPPORTED;
+    const AttnPlan plan = plan_attn(p, rows, items_per_row);
+    if (plan.bytes() > ws_bytes) return CSA_ERR_WORKSPACE;
+    if (plan.bytes() && !ws) return CSA_ERR_ARG;
+    AttnArgs a;
+    a.H = p->n_heads; a.D = p->head_dim; a.m = p->m; a.W = p->window; a.k = p->top_k;
+    a.scale = p->scale;
+    a.q = q; a.kv = kv; a.kv_s = kv_s; a.max_entries = max_entries; a.idx = idx;
+    a.raw = raw; a.n_raw = n_raw; a.raw_pos0 = raw_pos0; a.q_pos = q_pos; a.sinks = sinks;
+    a.n_q = n_q; a.n_splits = plan.n_splits; a.out = out;
+    a.part_o = (float*)ws;
+    a.part_ml = (float2*)((char*)ws + plan.part_o_bytes);
+    int st = cuda_status(launch_attn_simt(p->act_fmt, p->kv_fmt, a, rows, s));
+    if (st) return st;
+    if (plan.n_splits > 1)
+        st = cuda_status(launch_combine(p->act_fmt, p->n_heads, p->head_dim, plan.n_splits, rows,
+                                        a.part_o, a.part_ml, sinks, out, s));
+    return st;
+}
+
+__global__ void fill_positions_kernel(int64_t* q_pos, int64_t* pos0, int batch, int64_t T,
+                                      int64_t t0, int64_t raw_pos0) {
+    const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i < int64_t(batch) * T) q_pos[i] = t0 + i % T;
+    if (i < batch) pos0[i] = raw_pos0;
+}
+
+static cudaError_t launch_fill_positions(int64_t* q_pos, int64_t* pos0, int batch, int64_t T,
+                                         int64_t t0, int64_t raw_pos0, cudaStream_t s) {
+    const int64_t n = std::max<int64_t>(int64_t(batch) * T, batch);
+    fill_positions_kernel<<<unsigned(ceil_div(n, 256)), 256, 0, s>>>(q_pos, pos0, batch, T, t0, raw_pos0);
+    return cudaGetLastError();
+}
+
+static int check_attn_ptrs(const void* q, const void* kv, const void* kv_s, int kv_fmt,
+                           const void* raw, int64_t n_raw, const int64_t* raw_pos0,
+                           const int64_t* q_pos, void* out) {
+    if (!q || !kv || !q_pos || !out || !raw_pos0) return CSA_ERR_ARG;
+    if (n_raw < 0 || (n_raw > 0 && !raw)) return CSA_ERR_ARG;
+    if (kv_fmt == CSA_FP8_S64 && !kv_s) return CSA_ERR_ARG;
+    if (!aligned16(q) || !aligned16(kv) || !aligned16(kv_s) || !aligned16(raw) || !aligned16(out))
+        return CSA_ERR_ALIGN;
+    return CSA_OK;
+}
+
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" {
+
+int csa_compress(const csa_params* p, int32_t d, const void* x, const void* z, const float* bias,
+                 int64_t n_tokens, int32_t out_fmt, void* out, void* out_scales,
+                 csa_stream_t stream) {
+    if (!p || p->m <= 0 || d <= 0 || (d % 64) != 0 || n_tokens < 0 || (n_tokens % p->m) != 0)
+        return CSA_ERR_ARG;
+    if (!act_ok(p->act_fmt)) return CSA_ERR_ARG;
+    if (out_fmt < CSA_F32 || out_fmt > CSA_MXFP4) return CSA_ERR_ARG;
+    if (n_tokens == 0) return CSA_OK;
+    if (!x || !z || !bias || !out) return CSA_ERR_ARG;
+    if ((out_fmt == CSA_FP8_S64 || out_fmt == CSA_MXFP4) && !out_scales) return CSA_ERR_ARG;
+    if (!aligned16(x) || !aligned16(z) || !aligned16(bias) || !aligned16(out) || !aligned16(out_scales))
+        return CSA_ERR_ALIGN;
+    return cuda_status(launch_compress(p->act_fmt, out_fmt, x, z, bias, n_tokens, p->m, d, out,
+                                       out_scales, (cudaStream_t)stream));
+}
+
+int csa_quantize(int32_t fmt, const float* src, int64_t rows, int32_t d, void* out,
+                 void* out_scales, csa_stream_t stream) {
+    if (d <= 0 || (d % 64) != 0 || rows < 0) return CSA_ERR_ARG;
+    if (fmt != CSA_BF16 && fmt != CSA_FP8_S64 && fmt != CSA_MXFP4 && fmt != CSA_F32) return CSA_ERR_ARG;
+    if (rows == 0) return CSA_OK;
+    if (!src || !out || (fmt >= CSA_FP8_S64 && !out_scales)) return CSA_ERR_ARG;
+    if (!aligned16(src) || !aligned16(out) || !aligned16(out_scales)) return CSA_ERR_ALIGN;
+    return cuda_status(launch_quantize(fmt, src, rows, d, out, out_scales, (cudaStream_t)stream));
+}
+
+int indexer_score(const csa_params* p, int32_t batch, int32_t n_q, const void* qI,
+                  const void* qI_scales, const float* w, const void* kI, const void* kI_scales,
+                  int64_t max_blocks, const int64_t* q_pos, float* scores, int64_t ld_scores,
+                  csa_stream_t stream) {
+    int st = check_params(p, true, false);
+    if (st) return st;
+    if (batch < 0 || n_q < 0 || max_blocks < 0 || ld_scores < max_blocks) return CSA_ERR_ARG;
+    if (batch == 0 || n_q == 0 || max_blocks == 0) return CSA_OK;
+    if (!qI || !w || !kI || !q_pos || !scores) return CSA_ERR_ARG;
+    if (p->idx_fmt == CSA_MXFP4 && (!qI_scales || !kI_scales)) return CSA_ERR_ARG;
+    if (!aligned16(qI) || !aligned16(kI) || !aligned16(scores)) return CSA_ERR_ALIGN;
+    return cuda_status(launch_indexer_simt(p->idx_fmt, p->idx_heads, p->idx_dim, p->m, p->window,
+                                           qI, qI_scales, w, kI, kI_scales, max_blocks, q_pos,
+                                           batch, n_q, max_blocks, scores, ld_scores,
+                                           (cudaStream_t)stream));
+}
+
+int topk_select(const csa_params* p, int32_t batch, int32_t n_q, const float* scores,
+                int64_t ld_scores, int64_t max_blocks, const int64_t* q_pos, int32_t* idx,
+                csa_stream_t stream) {
+    if (!p || p->m <= 0 || p->window < 0 || p->top_k <= 0) return CSA_ERR_ARG;
+    if (batch < 0 || n_q < 0 || max_blocks < 0 || ld_scores < max_blocks) return CSA_ERR_ARG;
+    if (max_blocks > INT32_MAX) return CSA_ERR_UNSUPPORTED;
+    if (batch == 0 || n_q == 0) return CSA_OK;
+    if (!q_pos || !idx || (max_blocks > 0 && !scores)) return CSA_ERR_ARG;
+    return cuda_status(launch_topk(scores, ld_scores, max_blocks, q_pos, p->m, p->window, p->top_k,
+                                   int64_t(batch) * n_q, idx, (cudaStream_t)stream));
+}
+
+int sparse_mqa_attn(const csa_params* p, int32_t batch, int32_t n_q, const void* q, const void* kv,
+                    const void* kv_scales, int64_t max_entries, const int32_t* idx,
+                    const void* raw, int64_t n_raw, const int64_t* raw_pos0,
+                    const int64_t* q_pos, const float* sinks, void* out, void* workspace,
+                    size_t ws_bytes, csa_stream_t stream) {
+    int st = check_params(p, false, true);
+    if (st) return st;
+    if (p->top_k <= 0 || batch < 0 || n_q < 0 || max_entries < 0) return CSA_ERR_ARG;
+    if (batch == 0 || n_q == 0) return CSA_OK;
+    if (!idx) return CSA_ERR_ARG;
+    st = check_attn_ptrs(q, kv, kv_scales, p->kv_fmt, raw, n_raw, raw_pos0, q_pos, out);
+    if (st) return st;
+    return run_attn(p, batch, n_q, q, kv, kv_scales, max_entries, idx, raw, n_raw, raw_pos0, q_pos,
+                    sinks, out, workspace, ws_bytes, int64_t(p->top_k) + p->window,
+                    (cudaStream_t)stream);
+}
+
+int hca_attn(const csa_params* p, int32_t batch, int32_t n_q, const void* q, const void* kv,
+             const void* kv_scales, int64_t max_entries, const void* raw, int64_t n_raw,
+             const int64_t* raw_pos0, const int64_t* q_pos, const float* sinks, void* out,
+             void* workspace, size_t ws_bytes, csa_stream_t stream) {
+    int st = check_params(p, false, true);
+    if (st) return st;
+    if (batch < 0 || n_q < 0 || max_entries < 0) return CSA_ERR_ARG;
+    if (batch == 0 || n_q == 0) return CSA_OK;
+    st = check_attn_ptrs(q, kv, kv_scales, p->kv_fmt, raw, n_raw, raw_pos0, q_pos, out);
+    if (st) return st;
+    return run_attn(p, batch, n_q, q, kv, kv_scales, max_entries, nullptr, raw, n_raw, raw_pos0,
+                    q_pos, sinks, out, workspace, ws_bytes, max_entries + p->window,
+                    (cudaStream_t)stream);
+}
+
+size_t csa_workspace_size(const csa_params* p, int32_t op, int32_t batch, int64_t n_q,
+                          int64_t n_ctx) {
+    if (!p || batch < 0 || n_q < 0 || n_ctx < 0 || p->n_heads <= 0 || p->head_dim <= 0) return 0;
+    const int64_t rows = int64_t(batch) * n_q;
+    switch (op) {
+    case CSA_OP_SPARSE_ATTN:
+        return plan_attn(p, rows, int64_t(p->top_k) + p->window).bytes() + 256;
+    case CSA_OP_HCA_ATTN:
+        return plan_attn(p, rows, n_ctx + p->window).bytes() + 256;
+    case CSA_OP_DECODE:
+    case CSA_OP_PREFILL: {
+        const size_t pos = op == CSA_OP_PREFILL ? ((size_t(rows) + batch) * 8 + 255) & ~size_t(255) : 0;
+        const size_t scores = ((size_t(rows) * size_t(std::max<int64_t>(n_ctx, 1)) * 4) + 255) & ~size_t(255);
+        const size_t sel = ((size_t(rows) * p->top_k * 4) + 255) & ~size_t(255);
+        return pos + scores + sel + plan_attn(p, rows, int64_t(p->top_k) + p->window).bytes() + 256;
+    }
+    default:
+        return 0;
+    }
+}
+
+int csa_decode(const csa_params* p, int32_t batch, const void* q, const void* qI,
+               const void* qI_scales, const float* w, const void* kv, const void* kv_scales,
+               const void* kI, const void* kI_scales, int64_t max_blocks, const void* raw,
+               int64_t n_raw, const int64_t* raw_pos0, const int64_t* q_pos, const float* sinks,
+               void* out, int32_t* idx_out, void* workspace, size_t ws_bytes,
+               csa_stream_t stream) {
+    int st = check_params(p, true, true);
+    if (st) return st;
+    if (batch < 0 || max_blocks < 0) return CSA_ERR_ARG;
+    if (batch == 0) return CSA_OK;
+    if (!workspace) return CSA_ERR_ARG;
+    if (ws_bytes < csa_workspace_size(p, CSA_OP_DECODE, batch, 1, max_blocks)) return CSA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return CSA_ERR_ALIGN;
+    const int64_t ld = std::max<int64_t>(max_blocks, 1);
+    float* scores = (float*)workspace;
+    const size_t sc_bytes = ((size_t(batch) * ld * 4) + 255) & ~size_t(255);
+    int32_t* sel = idx_out ? idx_out : (int32_t*)((char*)workspace + sc_bytes);
+    const size_t sel_bytes = ((size_t(batch) * p->top_k * 4) + 255) & ~size_t(255);
+    void* ws_attn = (char*)workspace + sc_bytes + sel_bytes;
+    const size_t ws_attn_bytes = ws_bytes - sc_bytes - sel_bytes;
+    cudaStream_t s = (cudaStream_t)stream;
+    st = indexer_score(p, batch, 1, qI, qI_scales, w, kI, kI_scales, max_blocks, q_pos, scores, ld,
+                       stream);
+    if (st) return st;
+    st = topk_select(p, batch, 1, scores, ld, max_blocks, q_pos, sel, stream);
+    if (st) return st;
+    return sparse_mqa_attn(p, batch, 1, q, kv, kv_scales, max_blocks, sel, raw, n_raw, raw_pos0,
+                           q_pos, sinks, out, ws_attn, ws_attn_bytes, stream);
+    (void)s;
+}
+
+int csa_prefill(const csa_params* p, int32_t batch, int64_t T, int64_t t0, const void* raw,
+                int64_t n_raw, int64_t raw_pos0, const void* z, const float* bias, const void* q,
+                const void* qI, const void* qI_scales, const float* w, void* kv, void* kv_scales,
+                const void* kI, const void* kI_scales, int64_t max_blocks, const float* sinks,
+                void* out, int32_t* idx_out, void* workspace, size_t ws_bytes,
+                csa_stream_t stream) {
+    int st = check_params(p, true, true);
+    if (st) return st;
+    if (batch < 0 || T < 0 || t0 < 0 || (t0 % p->m) != 0 || max_blocks < 0) return CSA_ERR_ARG;
+    if (batch == 0 || T == 0) return CSA_OK;
+    if (!raw || !z || !bias || !kv || !workspace) return CSA_ERR_ARG;
+    if (T > INT32_MAX) return CSA_ERR_UNSUPPORTED;
+    // the chunk's tokens must be in the raw buffer; the window needs the W-1 before it
+    if (raw_pos0 > t0 || raw_pos0 + n_raw < t0 + T) return CSA_ERR_ARG;
+    if (raw_pos0 > std::max<int64_t>(0, t0 - p->window + 1)) return CSA_ERR_ARG;
+    const int64_t nb_end = (t0 + T) / p->m;  // pooled entries after the chunk
+    if (nb_end > max_blocks) return CSA_ERR_ARG;
+    if (ws_bytes < csa_workspace_size(p, CSA_OP_PREFILL, batch, T, max_blocks)) return CSA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return CSA_ERR_ALIGN;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t rows = int64_t(batch) * T;
+    const int64_t ld = std::max<int64_t>(max_blocks, 1);
+    char* wp = (char*)workspace;
+    int64_t* q_pos = (int64_t*)wp;
+    wp += ((size_t(rows) + size_t(batch)) * 8 + 255) & ~size_t(255);
+    int64_t* pos0 = q_pos + rows;
+    float* scores = (float*)wp;
+    wp += ((size_t(rows) * ld * 4) + 255) & ~size_t(255);
+    int32_t* sel = idx_out ? idx_out : (int32_t*)wp;
+    wp += ((size_t(rows) * p->top_k * 4) + 255) & ~size_t(255);
+    const size_t used = size_t(wp - (char*)workspace);
+    st = cuda_status(launch_fill_positions(q_pos, pos0, batch, T, t0, raw_pos0, s));
+    if (st) return st;
+    // 1. pool the chunk's complete blocks into kv entries [t0/m, (t0+T)/m)
+    const int64_t n_pool = (T / p->m) * p->m;
+    const size_t act_es = p->act_fmt == CSA_F32 ? 4 : 2;
+    const size_t kv_es = p->kv_fmt == CSA_F32 ? 4 : (p->kv_fmt == CSA_BF16 ? 2 : 1);
+    const int d = p->head_dim;
+    for (int b = 0; b < batch && n_pool > 0; ++b) {
+        const char* xb = (const char*)raw + (size_t(b) * n_raw + size_t(t0 - raw_pos0)) * d * act_es;
+        const char* zb = (const char*)z + size_t(b) * T * d * act_es;
+        char* ob = (char*)kv + (size_t(b) * max_blocks + size_t(t0 / p->m)) * d * kv_es;
+        char* osb = nullptr;
+        if (p->kv_fmt == CSA_FP8_S64) {
+            if (!kv_scales) return CSA_ERR_ARG;
+            osb = (char*)kv_scales + (size_t(b) * max_blocks + size_t(t0 / p->m)) * (d / 64) * 4;
+        }
+        st = csa_compress(p, d, xb, zb, bias, n_pool, p->kv_fmt, ob, osb, stream);
+        if (st) return st;
+    }
+    // 2-4. score, select, attend
+    st = indexer_score(p, batch, int32_t(T), qI, qI_scales, w, kI, kI_scales, max_blocks, q_pos,
+                       scores, ld, stream);
+    if (st) return st;
+    st = topk_select(p, batch, int32_t(T), scores, ld, max_blocks, q_pos, sel, stream);
+    if (st) return st;
+    return sparse_mqa_attn(p, batch, int32_t(T), q, kv, kv_scales, max_blocks, sel, raw, n_raw,
+                           pos0, q_pos, sinks, out, wp, ws_bytes - used, stream);
+}
+
+int csa_device_status(csa_stream_t stream, uint32_t* flags, int32_t reset) {
+    if (!flags) return CSA_ERR_ARG;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return CSA_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return CSA_ERR_CUDA;
+    *flags = v;
+    if (reset) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return CSA_ERR_CUDA;
+    }
+    return CSA_OK;
+}
+
+const char* csa_strerror(int status) {
+    switch (status) {
+    case CSA_OK: return "ok";
+    case CSA_ERR_ARG: return "invalid argument";
+    case CSA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case CSA_ERR_UNSUPPORTED: return "shape or format combination not supported";
+    case CSA_ERR_WORKSPACE: return "workspace too small";
+    case CSA_ERR_CUDA: return "CUDA launch failed";
+    default: return "unknown status";
+    }
+}
+
+const char* csa_version(void) { return "csa13 0.1.0 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,162 @@
+// Softmax-gated pooling of m tokens into one entry, and the store of fp32
+// rows as FP8 (E4M3 + fp32 scale per 64 channels), MXFP4 (E2M1 + E8M0 per
+// 32 channels) or bf16.
+//
+// Pooling ("DeepSeek-V4 發佈說明", sections 壓縮稀疏注意力 (CSA) and 重度壓縮注意力
+// (HCA)): per channel c, the m tokens of block j are weighted by a softmax
+// over the slots of z + B[slot], then summed.  FP8 entries and an FP4
+// indexer are the storage formats named in section 架構實現.
+//
+// One warp owns one 64-channel group of one output row: each lane holds two
+// adjacent channels, so every load is a coalesced 256 B (fp32) or 128 B
+// (bf16) row segment, the FP8 scale group is exactly one warp and an MXFP4
+// block is one half-warp.  The pass over the m slots reads z twice (max,
+// then exp-sum) so each weight is a single exp; the kernel is HBM-bound on
+// the x / z reads.
+#include "kernels.h"
+
+namespace csa {
+
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+    uint16_t r;
+    asm("{ .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n mov.b16 %0, {t, 0}; }"
+        : "=h"(r)
+        : "f"(hi), "f"(lo));
+    return r & 0xFFu;
+}
+
+// 2^e as a float for e in [-127, 127] (exact).
+__device__ __forceinline__ float pow2f(int e) {
+    return e >= -126 ? __int_as_float((e + 127) << 23) : __int_as_float(0x00400000);
+}
+
+template <int FMT>
+__device__ __forceinline__ float2 load_pair(const void* p, int64_t off) {
+    if constexpr (FMT == CSA_F32) {
+        return *reinterpret_cast<const float2*>((const float*)p + off);
+    } else {
+        const uint32_t u = *reinterpret_cast<const uint32_t*>((const uint16_t*)p + off);
+        return make_float2(__int_as_float(int(u << 16)), __int_as_float(int(u & 0xFFFF0000u)));
+    }
+}
+
+// Store the pair (v0, v1) of channels (c, c+1) of row j in OUT_FMT.  All 32
+// lanes of the warp must call this together (group reductions).
+template <int OUT_FMT>
+__device__ __forceinline__ void store_pair(float v0, float v1, int64_t j, int d, int c, int lane,
+                                           void* out, void* out_scales) {
+    if constexpr (OUT_FMT == CSA_F32) {
+        *reinterpret_cast<float2*>((float*)out + j * d + c) = make_float2(v0, v1);
+    } else if constexpr (OUT_FMT == CSA_BF16) {
+        __nv_bfloat162 b = __floats2bfloat162_rn(v0, v1);
+        *reinterpret_cast<__nv_bfloat162*>((uint16_t*)out + j * d + c) = b;
+    } else if constexpr (OUT_FMT == CSA_FP8_S64) {
+        const float amax = warp_max(fmaxf(fabsf(v0), fabsf(v1)));
+        const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        const uint16_t codes = cvt_e4m3x2(__fdiv_rn(v0, scale), __fdiv_rn(v1, scale));
+        *reinterpret_cast<uint16_t*>((uint8_t*)out + j * d + c) = codes;
+        if (lane == 0) ((float*)out_scales)[j * (d / 64) + c / 64] = scale;
+    } else {  // MXFP4: a half-warp covers one 32-channel block
+        float a = fmaxf(fabsf(v0), fabsf(v1));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        int X = a > 0.f ? ilog2_floor(a) - 2 : 0;
+        X = max(-127, min(127, X));
+        const float inv = pow2f(-X);
+        const uint32_t byte = cvt_e2m1x2(__fmul_rn(v0, inv), __fmul_rn(v1, inv));
+        ((uint8_t*)out)[j * (d / 2) + c / 2] = (uint8_t)byte;
+        if ((lane & 15) == 0) ((uint8_t*)out_scales)[j * (d / 32) + c / 32] = (uint8_t)(X + 127);
+    }
+}
+
+// POOL: out row j pools input rows [j*m, j*m+m) with gate z + bias.
+// !POOL: out row j is input row j (a pure format conversion; m, z, bias unused).
+template <int IN_FMT, int OUT_FMT, bool POOL>
+__global__ void __launch_bounds__(256) pool_kernel(const void* __restrict__ x,
+                                                   const void* __restrict__ z,
+                                                   const float* __restrict__ bias, int64_t n_out,
+                                                   int m, int d, void* out, void* out_scales) {
+    const int64_t gw = int64_t(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x & 31;
+    const int groups = d / 64;
+    if (gw >= n_out * groups) return;  // whole warps exit together
+    const int64_t j = gw / groups;
+    const int c = int(gw % groups) * 64 + 2 * lane;
+    float v0, v1;
+    if constexpr (POOL) {
+        const int64_t r0 = j * m;
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+        for (int r = 0; r < m; ++r) {
+            const float2 zz = load_pair<IN_FMT>(z, (r0 + r) * d + c);
+            const float2 bb = *reinterpret_cast<const float2*>(bias + int64_t(r) * d + c);
+            mx0 = fmaxf(mx0, zz.x + bb.x);
+            mx1 = fmaxf(mx1, zz.y + bb.y);
+        }
+        float den0 = 0.f, den1 = 0.f, acc0 = 0.f, acc1 = 0.f;
+        for (int r = 0; r < m; ++r) {
+            const float2 zz = load_pair<IN_FMT>(z, (r0 + r) * d + c);
+            const float2 bb = *reinterpret_cast<const float2*>(bias + int64_t(r) * d + c);
+            const float2 xx = load_pair<IN_FMT>(x, (r0 + r) * d + c);
+            const float e0 = expf(zz.x + bb.x - mx0), e1 = expf(zz.y + bb.y - mx1);
+            den0 += e0;
+            den1 += e1;
+            acc0 = fmaf(e0, xx.x, acc0);
+            acc1 = fmaf(e1, xx.y, acc1);
+        }
+        v0 = acc0 / den0;
+        v1 = acc1 / den1;
+    } else {
+        const float2 xx = load_pair<IN_FMT>(x, j * d + c);
+        v0 = xx.x;
+        v1 = xx.y;
+    }
+    store_pair<OUT_FMT>(v0, v1, j, d, c, lane, out, out_scales);
+}
+
+template <int IN_FMT, bool POOL>
+static cudaError_t launch_pool_out(int out_fmt, const void* x, const void* z, const float* bias,
+                                   int64_t n_out, int m, int d, void* out, void* out_scales,
+                                   cudaStream_t s) {
+    const int64_t warps = n_out * (d / 64);
+    const dim3 grid(unsigned(ceil_div(warps, 8)));
+    switch (out_fmt) {
+    case CSA_F32:
+        pool_kernel<IN_FMT, CSA_F32, POOL><<<grid, 256, 0, s>>>(x, z, bias, n_out, m, d, out, out_scales);
+        break;
+    case CSA_BF16:
+        pool_kernel<IN_FMT, CSA_BF16, POOL><<<grid, 256, 0, s>>>(x, z, bias, n_out, m, d, out, out_scales);
+        break;
+    case CSA_FP8_S64:
+        pool_kernel<IN_FMT, CSA_FP8_S64, POOL><<<grid, 256, 0, s>>>(x, z, bias, n_out, m, d, out, out_scales);
+        break;
+    default:
+        pool_kernel<IN_FMT, CSA_MXFP4, POOL><<<grid, 256, 0, s>>>(x, z, bias, n_out, m, d, out, out_scales);
+        break;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_compress(int in_fmt, int out_fmt, const void* x, const void* z,
+                            const float* bias, int64_t n_tokens, int m, int d, void* out,
+                            void* out_scales, cudaStream_t s) {
+    const int64_t n_out = n_tokens / m;
+    if (n_out == 0) return cudaSuccess;
+    if (in_fmt == CSA_F32)
+        return launch_pool_out<CSA_F32, true>(out_fmt, x, z, bias, n_out, m, d, out, out_scales, s);
+    return launch_pool_out<CSA_BF16, true>(out_fmt, x, z, bias, n_out, m, d, out, out_scales, s);
+}
+
+cudaError_t launch_quantize(int out_fmt, const float* src, int64_t rows, int d, void* out,
+                            void* out_scales, cudaStream_t s) {
+    if (rows == 0) return cudaSuccess;
+    return launch_pool_out<CSA_F32, false>(out_fmt, src, nullptr, nullptr, rows, 1, d, out,
+                                           out_scales, s);
+}
+
+}  // namespace csa

@@ -1,0 +1,45 @@
+// Host-side launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+#include "common.cuh"
+
+namespace csa {
+
+// Arguments of the attention kernels (sparse CSA and dense HCA).
+struct AttnArgs {
+    int H, D, m, W, k;
+    float scale;
+    const void* q;          // [rows][H][D] act format
+    const void* kv;         // [batch][max_entries][D] kv format
+    const void* kv_s;       // scales of kv (FP8_S64) or null
+    int64_t max_entries;
+    const int32_t* idx;     // [rows][k] selected ids, or null for dense (HCA)
+    const void* raw;        // [batch][n_raw][D] act format
+    int64_t n_raw;
+    const int64_t* raw_pos0;  // [batch]
+    const int64_t* q_pos;     // [rows]
+    const float* sinks;       // [H] or null
+    int n_q;                  // queries per sequence (row = b * n_q + i)
+    int n_splits;
+    void* out;                // final output when n_splits == 1
+    float* part_o;            // [rows][n_splits][H][D]
+    float2* part_ml;          // [rows][n_splits][H] (running max, running sum)
+};
+
+cudaError_t launch_compress(int in_fmt, int out_fmt, const void* x, const void* z,
+                            const float* bias, int64_t n_tokens, int m, int d, void* out,
+                            void* out_scales, cudaStream_t s);
+cudaError_t launch_quantize(int out_fmt, const float* src, int64_t rows, int d, void* out,
+                            void* out_scales, cudaStream_t s);
+cudaError_t launch_indexer_simt(int fmt, int HI, int dI, int m, int W, const void* qI,
+                                const void* qI_s, const float* w, const void* kI,
+                                const void* kI_s, int64_t max_blocks, const int64_t* q_pos,
+                                int batch, int n_q, int64_t max_elig, float* scores, int64_t ld,
+                                cudaStream_t s);
+cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, const int64_t* q_pos,
+                        int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s);
+cudaError_t launch_attn_simt(int act, int kvf, const AttnArgs& a, int64_t rows, cudaStream_t s);
+bool attn_simt_supported(int act, int kvf, int H, int D);
+cudaError_t launch_combine(int act, int H, int D, int n_splits, int64_t rows, const float* part_o,
+                           const float2* part_ml, const float* sinks, void* out, cudaStream_t s);
+
+}  // namespace csa

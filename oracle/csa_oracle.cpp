@@ -266,11 +266,15 @@ int64_t orc_n_elig(int64_t t, int m, int W) { return n_elig(t, m, W); }
 // row q_row; w: [HI]; keys: rows [0, n) of `kv`.  scores: fp32 [n].
 static void indexer_row(const View& qv, int64_t q_row, const float* w, const View& kv,
                         int64_t n, int HI, int dI, float* scores) {
+    std::vector<double> q(size_t(HI) * dI), k(dI);
+    for (int h = 0; h < HI; ++h)
+        for (int i = 0; i < dI; ++i) q[size_t(h) * dI + i] = view_get(qv, q_row + h, i);
     for (int64_t j = 0; j < n; ++j) {
+        for (int i = 0; i < dI; ++i) k[i] = view_get(kv, j, i);
         double s = 0;
         for (int h = 0; h < HI; ++h) {
             double dot = 0;
-            for (int i = 0; i < dI; ++i) dot += view_get(qv, q_row + h, i) * view_get(kv, j, i);
+            for (int i = 0; i < dI; ++i) dot += q[size_t(h) * dI + i] * k[i];
             s += double(w[h]) * std::max(0.0, dot);
         }
         scores[j] = float(s);
@@ -322,15 +326,19 @@ static void attend_row(const View& qv, int64_t q_row, int H, int d, double scale
                        const View& kv, const int64_t* ent, int64_t n_ent,
                        const View& rv, int64_t raw_lo, int64_t raw_hi,
                        const float* sinks, double* out) {
-    int64_t n = n_ent + std::max<int64_t>(0, raw_hi - raw_lo);
-    std::vector<double> logit(n);
-    std::vector<double> qh(d);
+    const int64_t n = n_ent + std::max<int64_t>(0, raw_hi - raw_lo);
+    // decode every attended item once: the key and the value of item e
+    std::vector<double> item(size_t(n) * d);
+    for (int64_t e = 0; e < n; ++e)
+        for (int c = 0; c < d; ++c)
+            item[size_t(e) * d + c] = e < n_ent ? view_get(kv, ent[e], c)
+                                                : view_get(rv, raw_lo + (e - n_ent), c);
+    std::vector<double> logit(n), qh(d);
     for (int h = 0; h < H; ++h) {
         for (int c = 0; c < d; ++c) qh[c] = view_get(qv, q_row + h, c);
         for (int64_t e = 0; e < n; ++e) {
             double dot = 0;
-            if (e < n_ent) for (int c = 0; c < d; ++c) dot += qh[c] * view_get(kv, ent[e], c);
-            else for (int c = 0; c < d; ++c) dot += qh[c] * view_get(rv, raw_lo + (e - n_ent), c);
+            for (int c = 0; c < d; ++c) dot += qh[c] * item[size_t(e) * d + c];
             logit[e] = scale * dot;
         }
         double M = sinks ? double(sinks[h]) : -INFINITY;
@@ -342,8 +350,7 @@ static void attend_row(const View& qv, int64_t q_row, int H, int d, double scale
         for (int64_t e = 0; e < n; ++e) {
             double p = std::exp(logit[e] - M);
             den += p;
-            if (e < n_ent) for (int c = 0; c < d; ++c) o[c] += p * view_get(kv, ent[e], c);
-            else for (int c = 0; c < d; ++c) o[c] += p * view_get(rv, raw_lo + (e - n_ent), c);
+            for (int c = 0; c < d; ++c) o[c] += p * item[size_t(e) * d + c];
         }
         for (int c = 0; c < d; ++c) o[c] /= den;
     }

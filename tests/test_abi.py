@@ -1,0 +1,103 @@
+"""The C-ABI library: it loads without a GPU, exports every symbol the header
+declares, and rejects bad arguments on the host before launching anything."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import compressed_sparse_attention_13_b200 as K
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", src, re.M):
+            if m.group(1) not in ("if", "sizeof", "defined"):
+                names.add(m.group(1))
+    return names
+
+
+def test_header_declares_the_entry_points():
+    want = {"csa_compress", "csa_quantize", "indexer_score", "topk_select", "sparse_mqa_attn",
+            "hca_attn", "csa_decode", "csa_prefill", "csa_workspace_size", "csa_device_status",
+            "csa_strerror", "csa_version"}
+    assert want <= _declared()
+
+
+def test_library_exports_every_declared_symbol():
+    lib = C.CDLL(K.LIB_PATH)
+    missing = [n for n in sorted(_declared()) if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(K.EXPORTS) <= _declared()
+
+
+def test_version_and_errors():
+    assert "sm_100a" in K.version()
+    for st in (0, -1, -2, -3, -4, -5):
+        assert K.strerror(st)
+    assert K.strerror(-99) == "unknown status"
+
+
+def test_workspace_size_contract():
+    p = K.params(4, 128, 512, 64, 512, 64, 128, 0.044)
+    assert K.csa_workspace_size(p, K.OP_DECODE, 32, 1, 32768) > 32 * 32768 * 4
+    assert K.csa_workspace_size(p, 99, 1, 1, 1) == 0
+    bad = K.params(4, 128, 512, 0, 512, 64, 128, 0.044)
+    assert K.csa_workspace_size(bad, K.OP_DECODE, 1, 1, 1) == 0
+
+
+def _call(fn, *args):
+    return getattr(K.lib(), fn)(*args)
+
+
+def test_host_side_argument_errors_need_no_gpu():
+    """Bad arguments are rejected before any CUDA call, so these run on CPU."""
+    lib = K.lib()
+    p = K.params(4, 128, 512, 64, 512, 64, 128, 0.044)
+    P = C.byref(p)
+    fake = C.c_void_p(0x1000)         # aligned, never dereferenced on the error paths
+    odd = C.c_void_p(0x1001)          # misaligned
+    # d not a multiple of 64
+    assert lib.csa_compress(P, 63, fake, fake, fake, 4, K.F32, fake, None, None) == -1
+    # token count not a multiple of m
+    assert lib.csa_compress(P, 64, fake, fake, fake, 6, K.F32, fake, None, None) == -1
+    # FP8 output without a scale buffer
+    assert lib.csa_compress(P, 64, fake, fake, fake, 8, K.FP8_S64, fake, None, None) == -1
+    # misaligned input
+    assert lib.csa_compress(P, 64, odd, fake, fake, 8, K.F32, fake, None, None) == -2
+    # unknown quantisation format
+    assert lib.csa_quantize(7, fake, 4, 64, fake, fake, None) == -1
+    # ld_scores smaller than max_blocks
+    assert lib.indexer_score(P, 1, 1, fake, fake, fake, fake, fake, 100, fake, fake, 50, None) == -1
+    # MXFP4 indexer without scales
+    assert lib.indexer_score(P, 1, 1, fake, None, fake, fake, None, 100, fake, fake, 100, None) == -1
+    # null selection for sparse attention
+    assert lib.sparse_mqa_attn(P, 1, 1, fake, fake, fake, 10, None, fake, 8, fake, fake, None,
+                               fake, fake, 1 << 30, None) == -1
+    # decode with a too-small workspace
+    assert lib.csa_decode(P, 32, fake, fake, fake, fake, fake, fake, fake, fake, 32768, fake, 128,
+                          fake, fake, None, fake, None, fake, 16, None) == -4
+    # prefill chunk start not a multiple of m
+    assert lib.csa_prefill(P, 1, 64, 3, fake, 64, 0, fake, fake, fake, fake, fake, fake, fake,
+                           fake, fake, fake, 100, None, fake, None, fake, 1 << 30, None) == -1
+    # bad parameter values
+    badp = K.params(0, 128, 512, 64, 512, 64, 128, 0.044)
+    assert lib.topk_select(C.byref(badp), 1, 1, fake, 10, 10, fake, fake, None) == -1
+    nanp = K.params(4, 128, 512, 64, 512, 64, 128, float("nan"))
+    assert lib.hca_attn(C.byref(nanp), 1, 1, fake, fake, fake, 10, fake, 8, fake, fake, None,
+                        fake, fake, 1 << 20, None) == -1
+
+
+def test_unbuilt_library_fails_loudly(monkeypatch, tmp_path):
+    import importlib
+    monkeypatch.setattr(K, "_lib", None)
+    monkeypatch.setattr(K, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        K.lib()

@@ -1,0 +1,278 @@
+"""Per-kernel parity of the CUDA library against the CPU oracle.
+
+Every test draws its inputs from the seeded generator, lets each side build
+its own stored tensors with its own quantiser, runs the library through the
+C ABI and the oracle on the CPU, and compares under the rules in helpers.py.
+Sizes are small enough for the oracle to finish in seconds but span several
+tiles and a ragged tail.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import compressed_sparse_attention_13_b200 as K
+import oracle
+import synth
+from helpers import (FMT, act_dev, act_orc, assert_close_abs, assert_close_f32, both_stored,
+                     check_selection, down, orc_quantize, quant_codes_match, up)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    K.csa_device_status(reset=True)
+    yield
+    assert K.csa_device_status(reset=True) == 0
+
+
+def _values(name, shape, seed=0, std=1.0):
+    return synth.tensor_np(seed, name, shape, std)
+
+
+# ---------------------------------------------------------------- quantisers
+@pytest.mark.parametrize("rows,d", [(1, 64), (37, 512), (300, 128)])
+def test_quantize_fp8_matches_oracle(rows, d):
+    v = _values("qf8", (rows, d))
+    v[0, :64] = 0.0
+    if rows > 2:
+        v[1, 3] = 1e5
+        v[2] *= 1e-6
+    g, o = both_stored(v, "fp8")
+    assert np.array_equal(down(g.scales), o.scales)
+    assert np.array_equal(down(g.data), o.data)
+
+
+@pytest.mark.parametrize("rows,d", [(1, 64), (33, 128), (300, 512)])
+def test_quantize_mxfp4_matches_oracle(rows, d):
+    v = _values("qf4", (rows, d))
+    v[0, :32] = 0.0
+    if rows > 2:
+        v[1] *= 1000.0
+        v[2, :32] = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0] * 4, np.float32)
+    g, o = both_stored(v, "mxfp4")
+    assert np.array_equal(down(g.scales), o.scales)
+    assert np.array_equal(down(g.data), o.data)
+
+
+def test_quantize_bf16_matches_oracle():
+    v = _values("qbf", (50, 128)) * 7
+    g, o = both_stored(v, "bf16")
+    assert np.array_equal(down(g.data), o.data)
+
+
+# ------------------------------------------------------------------- pooling
+@pytest.mark.parametrize("act,m,d,n_blocks,out", [
+    ("f32", 4, 64, 256, "f32"),
+    ("bf16", 4, 512, 97, "f32"),
+    ("bf16", 128, 512, 5, "f32"),
+    ("f32", 4, 128, 33, "f32"),
+])
+def test_compress_f32_out(act, m, d, n_blocks, out):
+    n = m * n_blocks
+    x = synth.tensor_np(1, "cx", (n, d), dtype=act)
+    z = synth.tensor_np(1, "cz", (n, d), dtype=act)
+    B = synth.tensor_np(1, "cb", (m, d), std=0.1)
+    p = K.params(m, 0, 1, 1, d, 1, 32, 1.0, act_fmt=FMT[act])
+    st = K.empty_stored(K.F32, n_blocks, d)
+    K.csa_compress(p, d, act_dev(x, act), act_dev(z, act), up(B), n, st)
+    ref = oracle.compress(act_orc(x, act), act_orc(z, act), B, m)
+    assert_close_f32(down(st.data), ref, 1e-5, "pooled entries")
+
+
+@pytest.mark.parametrize("act,m,d,n_blocks,fmt", [
+    ("bf16", 4, 512, 64, "fp8"),
+    ("bf16", 128, 512, 6, "fp8"),
+    ("bf16", 4, 512, 40, "bf16"),
+    ("f32", 4, 128, 70, "mxfp4"),
+])
+def test_compress_quantised_out(act, m, d, n_blocks, fmt):
+    n = m * n_blocks
+    x = synth.tensor_np(2, "cx", (n, d), dtype=act)
+    z = synth.tensor_np(2, "cz", (n, d), dtype=act)
+    B = synth.tensor_np(2, "cb", (m, d), std=0.1)
+    p = K.params(m, 0, 1, 1, d, 1, 32, 1.0, act_fmt=FMT[act])
+    st = K.empty_stored(FMT[fmt], n_blocks, d)
+    K.csa_compress(p, d, act_dev(x, act), act_dev(z, act), up(B), n, st)
+    pre = oracle.compress(act_orc(x, act), act_orc(z, act), B, m)
+    o = orc_quantize(pre, fmt)
+    if fmt == "bf16":
+        # both sides round their own fp32 value to bf16; the fp32 values agree
+        # within 1e-5 of the row magnitude, so the stored values may differ by
+        # one bf16 ulp where a value sits on a rounding boundary, or by that
+        # absolute error for values that cancel to near zero
+        g = synth.bf16_bits_to_f32_np(down(st.data)).astype(np.float64)
+        r = synth.bf16_bits_to_f32_np(o.data).astype(np.float64)
+        row = np.max(np.abs(pre), axis=1, keepdims=True)
+        tol = np.maximum(2.0 ** -8 * np.abs(r), 1e-5 * row)
+        assert (np.abs(g - r) <= tol).all(), np.max(np.abs(g - r) - tol)
+        return
+    gs = down(st.scales)
+    assert_close_f32(gs, o.scales, 1e-5, "scales")
+    if fmt == "fp8":
+        per_el = np.repeat(o.scales, 64, axis=1)
+        bad = quant_codes_match(down(st.data), o.data, pre, per_el, "fp8")
+    else:
+        assert np.array_equal(gs, o.scales)
+        per_el = np.repeat(2.0 ** (o.scales.astype(np.float64) - 127), 32, axis=1)
+        g_codes = down(st.data)
+        def unpack(a):
+            a = a.astype(np.uint8)
+            return np.stack([a & 15, a >> 4], -1).reshape(a.shape[0], -1)
+        bad = quant_codes_match(unpack(g_codes), unpack(o.data), pre, per_el, "mxfp4")
+    assert bad == 0
+
+
+# ------------------------------------------------------------------- indexer
+@pytest.mark.parametrize("idx,HI,dI,n_q,nb,m,W", [
+    ("f32", 4, 32, 40, 256, 4, 64),
+    ("bf16", 64, 128, 12, 700, 4, 128),
+    ("mxfp4", 64, 128, 3, 2100, 4, 128),
+])
+def test_indexer_matches_oracle(idx, HI, dI, n_q, nb, m, W):
+    batch = 2
+    qv = synth.tensor_np(3, "iq", (batch, n_q, HI, dI), dtype="f32" if idx != "bf16" else "bf16")
+    kv_ = synth.tensor_np(3, "ik", (batch, nb, dI), dtype="f32" if idx != "bf16" else "bf16")
+    w = synth.tensor_np(3, "iw", (batch, n_q, HI), std=0.1)
+    rng = np.random.default_rng(3)
+    q_pos = rng.integers(0, m * nb + W + 50, size=(batch, n_q)).astype(np.int64)
+    q_pos[0, 0] = m * nb + W + 10      # every block eligible
+    q_pos[1, 0] = 3                    # none eligible
+    p = K.params(m, W, 16, 1, 64, HI, dI, 1.0, idx_fmt=FMT[idx])
+    if idx == "bf16":
+        qd = K.Stored(K.BF16, up(qv, True))
+        kd = K.Stored(K.BF16, up(kv_, True))
+        qo = [oracle.Stored(oracle.BF16, qv[b].reshape(-1, dI)) for b in range(batch)]
+        ko = [oracle.Stored(oracle.BF16, kv_[b]) for b in range(batch)]
+    else:
+        qd, _ = both_stored(qv.reshape(-1, dI), idx)
+        kd, _ = both_stored(kv_.reshape(-1, dI), idx)
+        qo = [orc_quantize(qv[b].reshape(-1, dI), idx) for b in range(batch)]
+        ko = [orc_quantize(kv_[b], idx) for b in range(batch)]
+    scores = torch.full((batch, n_q, nb), float("nan"), device="cuda")
+    K.indexer_score(p, batch, n_q, qd, up(w), kd, nb, up(q_pos), scores, nb)
+    got = down(scores)
+    for b in range(batch):
+        ref = oracle.indexer(qo[b], w[b], ko[b], q_pos[b], HI, m, W)
+        qdq = oracle.dequantize(qo[b]).reshape(n_q, HI, dI)
+        kdq = oracle.dequantize(ko[b])
+        for i in range(n_q):
+            ne = min(oracle.n_elig(int(q_pos[b, i]), m, W), nb)
+            assert np.all(np.isnan(got[b, i, ne:])), "columns past n_elig must be untouched"
+            if ne == 0:
+                continue
+            # fp32 accumulation bound: 1e-5 of sum_h |w_h| |q_h| |k_j|
+            mag = (np.abs(w[b, i])[:, None] * np.linalg.norm(qdq[i], axis=1)[:, None] *
+                   np.linalg.norm(kdq[:ne], axis=1)[None, :]).sum(0)
+            err = np.abs(got[b, i, :ne] - ref[i, :ne])
+            assert (err <= 1e-5 * mag + 1e-30).all(), (b, i, err.max())
+
+
+# --------------------------------------------------------------------- top-k
+@pytest.mark.parametrize("n,k", [(50, 8), (2015, 512), (32736, 512), (5000, 1024)])
+def test_topk_matches_oracle_exactly(n, k):
+    rows = 6
+    s = synth.tensor_np(4, "ts", (rows, n))
+    s[1] = np.round(s[1] * 2) / 2          # many exact ties
+    s[2, ::3] = 0.0
+    s[2, 1::3] = -0.0                      # -0 and +0 are equal
+    s[3] = 0.25                            # all equal
+    m, W = 4, 128
+    q_pos = np.full(rows, m * n + W + 3, np.int64)
+    q_pos[4] = m * (k // 2) + W           # n_elig < k
+    q_pos[5] = m * k + W                  # n_elig == k
+    p = K.params(m, W, k, 1, 64, 1, 32, 1.0)
+    idx = torch.empty((rows, k), dtype=torch.int32, device="cuda")
+    K.topk_select(p, 1, rows, up(s), n, n, up(q_pos), idx)
+    ref = oracle.topk(s, q_pos, k, m, W)
+    assert np.array_equal(down(idx), ref)
+
+
+# ----------------------------------------------------------------- attention
+def _attn_case(act, kvf, H, d, batch, n_q, n_ent, W, k, m, seed, scale):
+    qv = synth.tensor_np(seed, "aq", (batch, n_q, H, d), dtype=act)
+    ent = synth.tensor_np(seed, "akv", (batch, n_ent, d))
+    n_raw = W + 40
+    raw = synth.tensor_np(seed, "araw", (batch, n_raw, d), dtype=act)
+    sinks = synth.tensor_np(seed, "asink", (H,))
+    rng = np.random.default_rng(seed)
+    t_hi = m * n_ent + W + 20
+    q_pos = rng.integers(0, t_hi, size=(batch, n_q)).astype(np.int64)
+    q_pos[:, 0] = t_hi
+    raw_pos0 = np.maximum(q_pos.max(1) - n_raw + 1, 0).astype(np.int64)
+    raw_pos0[0] = max(0, t_hi - W - 10)
+    return qv, ent, raw, n_raw, sinks, q_pos, raw_pos0
+
+
+@pytest.mark.parametrize("act,kvf,H,d,n_q,n_ent,W,k,m", [
+    ("f32", "f32", 8, 64, 20, 256, 64, 16, 4),
+    ("bf16", "fp8", 64, 512, 3, 700, 128, 512, 4),
+    ("bf16", "bf16", 64, 512, 4, 300, 128, 64, 4),
+])
+def test_sparse_attention_matches_oracle(act, kvf, H, d, n_q, n_ent, W, k, m):
+    batch, seed, scale = 2, 5, 1 / math.sqrt(d)
+    qv, ent, raw, n_raw, sinks, q_pos, raw_pos0 = _attn_case(act, kvf, H, d, batch, n_q, n_ent, W, k, m, seed, scale)
+    rng = np.random.default_rng(seed + 1)
+    idx = np.full((batch, n_q, k), -1, np.int32)
+    for b in range(batch):
+        for i in range(n_q):
+            ne = min(oracle.n_elig(int(q_pos[b, i]), m, W), n_ent)
+            c = np.sort(rng.permutation(ne)[:min(k, ne)])
+            idx[b, i, :len(c)] = c
+    kd, _ = both_stored(ent.reshape(-1, d), kvf)
+    p = K.params(m, W, k, H, d, 1, 32, scale, act_fmt=FMT[act], kv_fmt=FMT[kvf])
+    out = torch.empty((batch, n_q, H, d), dtype=torch.float32 if act == "f32" else torch.bfloat16,
+                      device="cuda")
+    ws = torch.empty(K.csa_workspace_size(p, K.OP_SPARSE_ATTN, batch, n_q, 0), dtype=torch.uint8,
+                     device="cuda")
+    K.sparse_mqa_attn(p, batch, n_q, act_dev(qv, act), kd, n_ent, up(idx), act_dev(raw, act),
+                      n_raw, up(raw_pos0), up(q_pos), up(sinks), out, ws)
+    got = down(out.float())
+    for b in range(batch):
+        ref = oracle.attention(act_orc(qv[b], act), orc_quantize(ent[b], kvf), idx[b],
+                               act_orc(raw[b], act), int(raw_pos0[b]), sinks, q_pos[b], H, m, W, scale)
+        if act == "f32":
+            assert_close_f32(got[b], ref, 1e-5, f"seq {b}")
+        else:
+            assert_close_abs(got[b], ref, 2e-2, f"seq {b}")
+
+
+@pytest.mark.parametrize("act,kvf,H,d,n_q,n_ent,W,m", [
+    ("f32", "f32", 8, 64, 10, 300, 64, 4),
+    ("bf16", "fp8", 64, 512, 2, 1500, 128, 128),
+])
+def test_hca_attention_matches_oracle(act, kvf, H, d, n_q, n_ent, W, m):
+    batch, seed, scale = 2, 6, 1 / math.sqrt(d)
+    qv, ent, raw, n_raw, sinks, q_pos, raw_pos0 = _attn_case(act, kvf, H, d, batch, n_q, n_ent, W, 0, m, seed, scale)
+    kd, _ = both_stored(ent.reshape(-1, d), kvf)
+    p = K.params(m, W, 1, H, d, 1, 32, scale, act_fmt=FMT[act], kv_fmt=FMT[kvf])
+    out = torch.empty((batch, n_q, H, d), dtype=torch.float32 if act == "f32" else torch.bfloat16,
+                      device="cuda")
+    ws = torch.empty(K.csa_workspace_size(p, K.OP_HCA_ATTN, batch, n_q, n_ent), dtype=torch.uint8,
+                     device="cuda")
+    K.hca_attn(p, batch, n_q, act_dev(qv, act), kd, n_ent, act_dev(raw, act), n_raw, up(raw_pos0),
+               up(q_pos), up(sinks), out, ws)
+    got = down(out.float())
+    for b in range(batch):
+        ref = oracle.attention(act_orc(qv[b], act), orc_quantize(ent[b], kvf), None,
+                               act_orc(raw[b], act), int(raw_pos0[b]), sinks, q_pos[b], H, m, W, scale)
+        if act == "f32":
+            assert_close_f32(got[b], ref, 1e-5, f"seq {b}")
+        else:
+            assert_close_abs(got[b], ref, 2e-2, f"seq {b}")
+
+
+def test_out_of_range_index_is_flagged_not_read():
+    H, d, m, W, k = 8, 64, 4, 4, 4
+    p = K.params(m, W, k, H, d, 1, 32, 0.125, act_fmt=K.F32, kv_fmt=K.F32)
+    q = torch.randn(1, 1, H, d, device="cuda")
+    kv = K.Stored(K.F32, torch.randn(10, d, device="cuda"))
+    idx = torch.tensor([[[0, 3, 1 << 20, -1]]], dtype=torch.int32, device="cuda")
+    raw = torch.randn(1, 8, d, device="cuda")
+    out = torch.empty(1, 1, H, d, device="cuda")
+    ws = torch.empty(K.csa_workspace_size(p, K.OP_SPARSE_ATTN, 1, 1, 0), dtype=torch.uint8, device="cuda")
+    K.sparse_mqa_attn(p, 1, 1, q, kv, 10, idx, raw, 8, up(np.array([0])), up(np.array([7])), None, out, ws)
+    assert K.csa_device_status(reset=True) == K.DEV_BAD_INDEX
+    assert torch.isfinite(out).all()
