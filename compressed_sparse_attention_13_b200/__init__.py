@@ -18,7 +18,7 @@ from dataclasses import dataclass
 
 F32, BF16, FP8_S64, MXFP4 = 0, 1, 2, 3
 OP_SPARSE_ATTN, OP_HCA_ATTN, OP_DECODE, OP_PREFILL = 0, 1, 2, 3
-DEV_BAD_INDEX, DEV_RANGE = 0x1, 0x2
+DEV_BAD_INDEX, DEV_RANGE, DEV_TIMEOUT = 0x1, 0x2, 0x4
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libcsa13.so")

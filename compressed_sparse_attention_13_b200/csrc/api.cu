@@ -154,7 +154,13 @@ int indexer_score(const csa_params* p, int32_t batch, int32_t n_q, const void* q
     if (batch == 0 || n_q == 0 || max_blocks == 0) return CSA_OK;
     if (!qI || !w || !kI || !q_pos || !scores) return CSA_ERR_ARG;
     if (p->idx_fmt == CSA_MXFP4 && (!qI_scales || !kI_scales)) return CSA_ERR_ARG;
-    if (!aligned16(qI) || !aligned16(kI) || !aligned16(scores)) return CSA_ERR_ALIGN;
+    if (!aligned16(qI) || !aligned16(kI) || !aligned16(scores) || !aligned16(qI_scales) ||
+        !aligned16(kI_scales))
+        return CSA_ERR_ALIGN;
+    if (indexer_tc_supported(p->idx_fmt, p->idx_heads, p->idx_dim, max_blocks))
+        return cuda_status(launch_indexer_tc(qI, qI_scales, w, kI, kI_scales, max_blocks, q_pos,
+                                             batch, n_q, p->m, p->window, scores, ld_scores,
+                                             (cudaStream_t)stream));
     return cuda_status(launch_indexer_simt(p->idx_fmt, p->idx_heads, p->idx_dim, p->m, p->window,
                                            qI, qI_scales, w, kI, kI_scales, max_blocks, q_pos,
                                            batch, n_q, max_blocks, scores, ld_scores,

@@ -35,6 +35,11 @@ cudaError_t launch_indexer_simt(int fmt, int HI, int dI, int m, int W, const voi
                                 const void* kI_s, int64_t max_blocks, const int64_t* q_pos,
                                 int batch, int n_q, int64_t max_elig, float* scores, int64_t ld,
                                 cudaStream_t s);
+bool indexer_tc_supported(int fmt, int HI, int dI, int64_t max_blocks);
+cudaError_t launch_indexer_tc(const void* qI, const void* qI_s, const float* w, const void* kI,
+                              const void* kI_s, int64_t max_blocks, const int64_t* q_pos,
+                              int batch, int n_q, int m, int W, float* scores, int64_t ld,
+                              cudaStream_t s);
 cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, const int64_t* q_pos,
                         int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s);
 cudaError_t launch_attn_simt(int act, int kvf, const AttnArgs& a, int64_t rows, cudaStream_t s);

@@ -4,9 +4,10 @@
 // memory and instruction descriptors the MMA reads.  Written from the PTX ISA
 // description of these instructions.
 //
-// Every wait on an mbarrier gives up after kSpinLimit polls, records
-// CSA_DEV_TIMEOUT in the device status word and reports failure, so that a
-// logic error ends the kernel instead of hanging the GPU.
+// Every wait on an mbarrier gives up after about kWaitNs nanoseconds of wall
+// time (read from %globaltimer), records CSA_DEV_TIMEOUT in the device status
+// word and reports failure, so that a logic error ends the kernel instead of
+// hanging the GPU.  Callers stop waiting after the first failure.
 #pragma once
 
 #include "common.cuh"
@@ -14,7 +15,13 @@
 namespace csa {
 namespace sm100 {
 
-constexpr uint32_t kSpinLimit = 1u << 26;  // polls (~0.5-1 s) before a wait gives up
+constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -54,10 +61,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and
-// flags CSA_DEV_TIMEOUT) if it does not within kSpinLimit polls.
+// flags CSA_DEV_TIMEOUT) if it does not within kWaitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 0 && global_ns() - t0 > kWaitNs) break;
+    }
     flag_status(CSA_DEV_TIMEOUT);
     return false;
 }

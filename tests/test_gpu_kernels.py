@@ -276,3 +276,19 @@ def test_out_of_range_index_is_flagged_not_read():
     K.sparse_mqa_attn(p, 1, 1, q, kv, 10, idx, raw, 8, up(np.array([0])), up(np.array([7])), None, out, ws)
     assert K.csa_device_status(reset=True) == K.DEV_BAD_INDEX
     assert torch.isfinite(out).all()
+
+
+def test_mxfp4_scale_outside_exact_range_is_flagged():
+    """The tensor-core indexer converts E2M1 x 2^X to E4M3 exactly only for X
+    in [-8, 6]; a larger block exponent must raise CSA_DEV_RANGE."""
+    HI, dI, nb, m, W = 64, 128, 256, 4, 128
+    qv = synth.tensor_np(8, "rq", (1, 1, HI, dI))
+    kv_ = synth.tensor_np(8, "rk", (1, nb, dI)) * 1e4      # X around 11
+    w = synth.tensor_np(8, "rw", (1, 1, HI), std=0.1)
+    q_pos = np.array([[m * nb + W]], np.int64)
+    p = K.params(m, W, 16, 1, 64, HI, dI, 1.0, idx_fmt=K.MXFP4)
+    qd, _ = both_stored(qv.reshape(-1, dI), "mxfp4")
+    kd, _ = both_stored(kv_.reshape(-1, dI), "mxfp4")
+    scores = torch.zeros((1, 1, nb), device="cuda")
+    K.indexer_score(p, 1, 1, qd, up(w), kd, nb, up(q_pos), scores, nb)
+    assert K.csa_device_status(reset=True) & K.DEV_RANGE
