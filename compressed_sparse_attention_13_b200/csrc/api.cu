@@ -50,9 +50,19 @@ struct AttnPlan {
     size_t bytes() const { return n_splits > 1 ? part_o_bytes + part_ml_bytes : 0; }
 };
 
+// The tensor-core kernel runs one 217 KB CTA per SM, so its splits fill the
+// 148 SMs in a single wave with at least one 128-item tile per split.
+static int choose_splits_tc(int64_t rows, int64_t items_per_row) {
+    if (rows >= kNumSMs) return 1;
+    const int64_t s = std::min<int64_t>(kNumSMs / rows, ceil_div(items_per_row, 128));
+    return int(std::max<int64_t>(1, std::min<int64_t>(s, 64)));
+}
+
 static AttnPlan plan_attn(const csa_params* p, int64_t rows, int64_t items_per_row) {
     AttnPlan a;
-    a.n_splits = choose_splits(rows, items_per_row);
+    a.n_splits = attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim)
+                     ? choose_splits_tc(rows, items_per_row)
+                     : choose_splits(rows, items_per_row);
     const int64_t items = rows * a.n_splits;
     a.part_o_bytes = size_t(items) * p->n_heads * p->head_dim * sizeof(float);
     a.part_ml_bytes = size_t(items) * p->n_heads * sizeof(float2);
@@ -66,7 +76,8 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
                     const float* sinks, void* out, void* ws, size_t ws_bytes, int64_t items_per_row,
                     cudaStream_t s) {
     const int64_t rows = int64_t(batch) * n_q;
-    if (!attn_simt_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim))
+    if (!attn_simt_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim) &&
+        !attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim))
         return CSA_ERR_UNSUPPORTED;
     const AttnPlan plan = plan_attn(p, rows, items_per_row);
     if (plan.bytes() > ws_bytes) return CSA_ERR_WORKSPACE;
@@ -79,7 +90,8 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
     a.n_q = n_q; a.n_splits = plan.n_splits; a.out = out;
     a.part_o = (float*)ws;
     a.part_ml = (float2*)((char*)ws + plan.part_o_bytes);
-    int st = cuda_status(launch_attn_simt(p->act_fmt, p->kv_fmt, a, rows, s));
+    const bool tc = attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim);
+    int st = cuda_status(tc ? launch_attn_tc(a, rows, s) : launch_attn_simt(p->act_fmt, p->kv_fmt, a, rows, s));
     if (st) return st;
     if (plan.n_splits > 1)
         st = cuda_status(launch_combine(p->act_fmt, p->n_heads, p->head_dim, plan.n_splits, rows,
