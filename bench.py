@@ -11,7 +11,9 @@ under "hca_decode".
 
 Timing: W untimed steps, then K steps, each bracketed by CUDA events on the
 launching stream with an L2 flush (a 256 MB write) between steps outside the
-events; barrier + synchronize on both sides; max over ranks.  Multi-GPU runs
+events; barrier + synchronize on both sides; max over ranks.  The device-side
+step is the library call captured once in a CUDA graph and replayed (the way
+a decode loop runs it); the e2e number calls the library eagerly.  Multi-GPU runs
 are independent replicas (weak scaling): each rank decodes its own batch.
 The reference arm (--impl reference) is the CPU oracle on a bounded sample of
 the same workload.
@@ -176,6 +178,21 @@ def time_steps(fn, steps, warmup, flush, stream):
     return [a.elapsed_time(b) for a, b in ev]
 
 
+def graphed(fn):
+    """Capture fn (a sequence of library calls on the current stream) in a
+    CUDA graph after one eager call; returns a replay function.  The decode
+    step is a handful of short launches, so host enqueue time would otherwise
+    show up as idle time inside the events."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g.replay
+
+
 def kernel_source_hash(files):
     h = hashlib.sha256()
     for f in files:
@@ -219,7 +236,8 @@ def run_ours(args):
     w = WORKLOADS[WORKLOAD]
     S = setup_csa_decode(w, dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    step = lambda: csa_decode_call(w, S)
+    eager_step = lambda: csa_decode_call(w, S)
+    step = graphed(eager_step)
 
     def barrier():
         if world > 1:
@@ -253,7 +271,7 @@ def run_ours(args):
     kfn["sparse_mqa_attn"] = lambda: K.sparse_mqa_attn(
         S["p"], w.batch, 1, S["q"], S["kv"], nb, S["sel"], S["window"], w.W, S["raw_pos0"],
         S["q_pos"], S["sinks"], S["out"], ws_attn)
-    kt = {name: statistics.mean(time_steps(fn, max(20, args.steps // 5), 3, flush, stream))
+    kt = {name: statistics.mean(time_steps(graphed(fn), max(20, args.steps // 5), 3, flush, stream))
           for name, fn in kfn.items()}
     by = csa_decode_bytes(w)
     idx_gbs = by["indexer"] / (kt["indexer_score"] / 1e3) / 1e9
@@ -272,7 +290,7 @@ def run_ours(args):
             S[n].copy_(host[n], non_blocking=True)
         S["qI"].data.copy_(host["qI"], non_blocking=True)
         S["qI"].scales.copy_(host["qI_s"], non_blocking=True)
-        step()
+        eager_step()
         out_h.copy_(S["out"], non_blocking=True)
 
     e2e_steps = max(10, args.steps // 5)
@@ -330,7 +348,7 @@ def bench_hca(args, dev, flush, stream, hbm_peak):
     x = draw_torch(w, "x", device=dev)
     z = draw_torch(w, "z", device=dev)
     comp = lambda: K.csa_compress(p, d, x, z, bias, B * N, kv)
-    t_comp = statistics.mean(time_steps(comp, 5, 1, flush, stream))
+    t_comp = statistics.mean(time_steps(graphed(comp), 5, 3, flush, stream))
     comp_bytes = 2 * B * N * d * 2 + B * nb * (d + 4 * d // 64)
     win = torch.cat([x[:, N - W + 1:], draw_torch(w, "x_new", device=dev)[:, None]], 1).contiguous()
     del x, z
@@ -339,7 +357,8 @@ def bench_hca(args, dev, flush, stream, hbm_peak):
     q_pos = torch.full((B,), N, dtype=torch.int64, device=dev)
     out = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
     ws = torch.empty(K.csa_workspace_size(p, K.OP_HCA_ATTN, B, 1, nb), dtype=torch.uint8, device=dev)
-    fn = lambda: K.hca_attn(p, B, 1, q, kv, nb, win, W, q_pos - W + 1, q_pos, sinks, out, ws)
+    raw_pos0 = q_pos - W + 1
+    fn = graphed(lambda: K.hca_attn(p, B, 1, q, kv, nb, win, W, raw_pos0, q_pos, sinks, out, ws))
     times = time_steps(fn, args.steps, args.warmup, flush, stream)
     t = statistics.mean(times)
     by = hca_decode_bytes(w)

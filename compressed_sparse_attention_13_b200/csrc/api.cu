@@ -2,11 +2,32 @@
 // host, workspace layout, and the choice of kernel for each format.
 #include <stdio.h>
 
+#include <mutex>
+
 #include "kernels.h"
 
 namespace csa {
 
 __device__ unsigned int g_status = 0;
+
+cudaError_t ensure_smem_impl(const void* kernel, size_t bytes) {
+    struct Entry { const void* k; int dev; size_t bytes; };
+    static Entry table[64];
+    static int used = 0;
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+        if (table[i].k == kernel && table[i].dev == dev && table[i].bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+    if (e != cudaSuccess) return e;
+    for (int i = 0; i < used; ++i)
+        if (table[i].k == kernel && table[i].dev == dev) { table[i].bytes = bytes; return e; }
+    if (used < 64) table[used++] = Entry{kernel, dev, bytes};
+    return e;
+}
 
 static bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 

@@ -103,4 +103,12 @@ __host__ __device__ __forceinline__ int64_t n_elig(int64_t t, int m, int W) {
 
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device): the
+// attribute call is host work that would otherwise sit between launches.
+cudaError_t ensure_smem_impl(const void* kernel, size_t bytes);
+template <typename K>
+inline cudaError_t ensure_smem(K* kernel, size_t bytes) {
+    return ensure_smem_impl(reinterpret_cast<const void*>(kernel), bytes);
+}
+
 }  // namespace csa

@@ -179,8 +179,7 @@ template <int DPT, int ACT, int KV>
 static cudaError_t launch_attn_t(const AttnArgs& a, int64_t rows, cudaStream_t s) {
     const size_t sm = size_t(a.H * a.D + kTile * (a.D + 1) + a.H * (kTile + 1) + 3 * a.H + 2) * 4 +
                       kTile * (8 + 4) + 16;
-    cudaError_t e = cudaFuncSetAttribute(attn_simt_kernel<DPT, ACT, KV>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
+    cudaError_t e = ensure_smem(attn_simt_kernel<DPT, ACT, KV>, size_t(sm));
     if (e != cudaSuccess) return e;
     attn_simt_kernel<DPT, ACT, KV><<<dim3(a.n_splits, unsigned(rows)), kAttnThreads, sm, s>>>(a);
     return cudaGetLastError();

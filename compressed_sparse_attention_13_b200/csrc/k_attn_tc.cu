@@ -28,6 +28,8 @@
 // softmax warps rescale O^T in TMEM before the next P.V product.
 // Bounded waits as in sm100.cuh; a role that timed out keeps iterating
 // through the named barriers without waiting.
+#include <type_traits>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -173,64 +175,94 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) 
         if (n_tiles > 0) {
             // query: 64 heads x 512 bf16 -> f16, K-major B tile (8 dim blocks)
             const uint16_t* qg = (const uint16_t*)a.q + row * int64_t(kH) * kD;
-            for (int u = pt; u < kH * (kD / 8); u += kProducerThreads) {
-                const int h = u >> 6, cc = u & 63;  // 8-dim chunk cc of head h
-                const uint4 v = *reinterpret_cast<const uint4*>(qg + h * kD + cc * 8);
-                const uint4 o = make_uint4(f16x2_of_bf16x2(v.x), f16x2_of_bf16x2(v.y),
-                                           f16x2_of_bf16x2(v.z), f16x2_of_bf16x2(v.w));
-                *reinterpret_cast<uint4*>(S.q[cc >> 3] + sw128_offset(h, cc & 7)) = o;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {  // 2 x 8 independent 16-byte loads per thread
+                uint4 v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int u = pt + kProducerThreads * (8 * half + j);
+                    v[j] = *reinterpret_cast<const uint4*>(qg + (u >> 6) * kD + (u & 63) * 8);
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int u = pt + kProducerThreads * (8 * half + j);
+                    const int h = u >> 6, cc = u & 63;  // 8-dim chunk cc of head h
+                    const uint4 o = make_uint4(f16x2_of_bf16x2(v[j].x), f16x2_of_bf16x2(v[j].y),
+                                               f16x2_of_bf16x2(v[j].z), f16x2_of_bf16x2(v[j].w));
+                    *reinterpret_cast<uint4*>(S.q[cc >> 3] + sw128_offset(h, cc & 7)) = o;
+                }
             }
             fence_proxy_async_smem();
             mbar_arrive(&S.q_full);
         }
-        bool ok = true;
-        for (int tile = 0; tile < n_tiles && ok; ++tile) {
-            Slot sl[8];
+        // Software pipeline over (tile, quarter) steps: the loads of step g+1
+        // are issued before step g waits for its buffer and converts, so two
+        // quarters of loads are in flight per thread.
+        const int n_steps = 4 * n_tiles;
+        int64_t src[8];  // source rows of this thread's 8 items in the tile being loaded
+        uint4 raw[2][8];
+        float sc[2][8];
+        // buffers are compile-time indices (the step loop is unrolled by two)
+        auto issue = [&](auto bufc, int g) {
+            constexpr int buf = decltype(bufc)::value;
+            const int tile = g >> 2, qt = g & 3;
+            const int64_t slot0 = s_lo + int64_t(tile) * kTileItems + (pt >> 4);
+            if (qt == 0) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                sl[i] = resolve_slot(a, row, b, n_kv, win_lo, s_lo + int64_t(tile) * kTileItems + (pt >> 4) + 16 * i, s_hi);
-            for (int qt = 0; qt < 4 && ok; ++qt) {
-                const int dim0 = 128 * qt + 8 * c;
-                uint4 raw[8];
-                float sc[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    raw[i] = make_uint4(0, 0, 0, 0);
-                    sc[i] = 0.f;
-                    if (sl[i].src >= 0) {
-                        if (sl[i].raw) {
-                            raw[i] = *reinterpret_cast<const uint4*>((const uint16_t*)a.raw + sl[i].src * kD + dim0);
-                        } else {
-                            const uint2 v = *reinterpret_cast<const uint2*>((const uint8_t*)a.kv + sl[i].src * kD + dim0);
-                            raw[i] = make_uint4(v.x, v.y, 0, 0);
-                            sc[i] = ((const float*)a.kv_s)[sl[i].src * (kD / 64) + (dim0 >> 6)];
-                        }
-                    }
-                }
-                if (tile > 0) ok = mbar_wait(&S.kv_empty[qt], uint32_t((tile - 1) & 1));
-                if (!ok) break;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int e = (pt >> 4) + 16 * i;
-                    uint4 o;
-                    if (sl[i].raw) {
-                        o = make_uint4(f16x2_of_bf16x2(raw[i].x), f16x2_of_bf16x2(raw[i].y),
-                                       f16x2_of_bf16x2(raw[i].z), f16x2_of_bf16x2(raw[i].w));
-                    } else {
-                        if (sc[i] != 0.f && (sc[i] < 6.103515625e-05f || sc[i] > 146.0f))
-                            flag_status(CSA_DEV_RANGE);
-                        const __half2 h2 = __float2half2_rn(sc[i]);
-                        const uint32_t s2 = *reinterpret_cast<const uint32_t*>(&h2);
-                        uint32_t f0, f1, f2, f3;
-                        f16x2_of_e4m3x4(raw[i].x, f0, f1);
-                        f16x2_of_e4m3x4(raw[i].y, f2, f3);
-                        o = make_uint4(hmul2(f0, s2), hmul2(f1, s2), hmul2(f2, s2), hmul2(f3, s2));
-                    }
-                    *reinterpret_cast<uint4*>(S.kv[2 * qt + (c >> 3)] + sw128_offset(e, c & 7)) = o;
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(&S.kv_full[qt]);
+                for (int i = 0; i < 8; ++i)
+                    src[i] = resolve_slot(a, row, b, n_kv, win_lo, slot0 + 16 * i, s_hi).src;
             }
+            const int dim0 = 128 * qt + 8 * c;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                raw[buf][i] = make_uint4(0, 0, 0, 0);
+                sc[buf][i] = 0.f;
+                if (src[i] >= 0) {
+                    if (slot0 + 16 * i >= n_kv) {  // a window token (bf16)
+                        raw[buf][i] = *reinterpret_cast<const uint4*>((const uint16_t*)a.raw + src[i] * kD + dim0);
+                    } else {
+                        const uint2 v = *reinterpret_cast<const uint2*>((const uint8_t*)a.kv + src[i] * kD + dim0);
+                        raw[buf][i] = make_uint4(v.x, v.y, 0, 0);
+                        sc[buf][i] = ((const float*)a.kv_s)[src[i] * (kD / 64) + (dim0 >> 6)];
+                    }
+                }
+            }
+        };
+        auto step = [&](auto bufc, int g) -> bool {
+            constexpr int buf = decltype(bufc)::value;
+            const int tile = g >> 2, qt = g & 3;
+            if (g + 1 < n_steps) issue(std::integral_constant<int, buf ^ 1>{}, g + 1);
+            if (tile > 0 && !mbar_wait(&S.kv_empty[qt], uint32_t((tile - 1) & 1))) return false;
+            const int64_t slot0 = s_lo + int64_t(tile) * kTileItems + (pt >> 4);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int e = (pt >> 4) + 16 * i;
+                uint4 o;
+                if (slot0 + 16 * i >= n_kv) {  // window token (or past the end: zeros either way)
+                    const uint4 r = raw[buf][i];
+                    o = make_uint4(f16x2_of_bf16x2(r.x), f16x2_of_bf16x2(r.y), f16x2_of_bf16x2(r.z),
+                                   f16x2_of_bf16x2(r.w));
+                } else {
+                    const float scl = sc[buf][i];
+                    if (scl != 0.f && (scl < 6.103515625e-05f || scl > 146.0f)) flag_status(CSA_DEV_RANGE);
+                    const __half2 h2 = __float2half2_rn(scl);
+                    const uint32_t s2 = *reinterpret_cast<const uint32_t*>(&h2);
+                    uint32_t f0, f1, f2, f3;
+                    f16x2_of_e4m3x4(raw[buf][i].x, f0, f1);
+                    f16x2_of_e4m3x4(raw[buf][i].y, f2, f3);
+                    o = make_uint4(hmul2(f0, s2), hmul2(f1, s2), hmul2(f2, s2), hmul2(f3, s2));
+                }
+                *reinterpret_cast<uint4*>(S.kv[2 * qt + (c >> 3)] + sw128_offset(e, c & 7)) = o;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&S.kv_full[qt]);
+            return true;
+        };
+        bool ok = true;
+        if (n_steps > 0) issue(std::integral_constant<int, 0>{}, 0);
+        for (int g = 0; g < n_steps && ok; g += 2) {
+            ok = step(std::integral_constant<int, 0>{}, g);
+            if (ok && g + 1 < n_steps) ok = step(std::integral_constant<int, 1>{}, g + 1);
         }
     } else if (warp == 12) {
         // --------------------------------------------------------------- MMA
@@ -416,7 +448,7 @@ bool attn_tc_supported(int act, int kvf, int H, int D) {
 cudaError_t launch_attn_tc(const AttnArgs& a, int64_t rows, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
     const size_t sm = sizeof(SmemAttn) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
+    cudaError_t e = ensure_smem(attn_tc_kernel, size_t(sm));
     if (e != cudaSuccess) return e;
     attn_tc_kernel<<<dim3(a.n_splits, unsigned(rows)), kThreads, sm, s>>>(a);
     return cudaGetLastError();

@@ -63,8 +63,7 @@ cudaError_t launch_indexer_simt(int fmt, int HI, int dI, int m, int W, const voi
     const size_t sm = size_t(HI * dI + 64 * (dI + 1) + 256) * sizeof(float);
     cudaError_t e;
 #define CSA_LAUNCH_IDX(F)                                                                          \
-    e = cudaFuncSetAttribute(indexer_simt_kernel<F>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             int(sm));                                                             \
+    e = ensure_smem(indexer_simt_kernel<F>, sm);                                                   \
     if (e != cudaSuccess) return e;                                                                \
     indexer_simt_kernel<F><<<grid, 256, sm, s>>>(HI, dI, m, W, qI, qI_s, w, kI, kI_s, max_blocks,  \
                                                  q_pos, n_q, scores, ld);

@@ -323,7 +323,7 @@ cudaError_t launch_indexer_tc(const void* qI, const void* qI_s, const float* w, 
     a.units = a.rows * a.tiles_per_row;
     if (a.units == 0) return cudaSuccess;
     const size_t sm = sizeof(Smem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
+    cudaError_t e = ensure_smem(indexer_tc_kernel, size_t(sm));
     if (e != cudaSuccess) return e;
     const int grid = int(std::min<int64_t>(kNumSMs, a.units));
     indexer_tc_kernel<<<grid, kThreads, sm, s>>>(a);

@@ -46,6 +46,50 @@ __device__ __forceinline__ int2 block_scan2(int2 v, int2* warp_tot) {
     return v;
 }
 
+// Output pass shared by both kernels: every key above T is taken, plus the
+// first `remaining` keys equal to T in index order; ids are written in
+// ascending order.  Warp w owns a contiguous segment of the row and walks it
+// 32 consecutive keys at a time (coalesced / bank-conflict free), compacting
+// with ballots; a block scan of the per-warp counts gives each warp its
+// output offset and its number of earlier equal keys.
+template <typename KeyAt>
+__device__ __forceinline__ void write_selection_impl(KeyAt key_at, int64_t n, uint32_t T, int remaining,
+                                                     int k, int32_t* out, int2* warp_tot) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    constexpr int kWarps = kTopkThreads / 32;
+    const int64_t seg = ((n + kWarps - 1) / kWarps + 31) / 32 * 32;
+    const int64_t lo = min(n, wid * seg), hi = min(n, lo + seg);
+    int gt = 0, eq = 0;
+    for (int64_t base = lo; base < hi; base += 32) {
+        const int64_t i = base + lane;
+        const uint32_t u = i < hi ? key_at(i) : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, i < hi && u > T));
+        eq += __popc(__ballot_sync(0xffffffffu, i < hi && u == T));
+    }
+    // exclusive scan over warps (lane 0 of each warp contributes)
+    const int2 inc = block_scan2(make_int2(lane == 0 ? gt : 0, lane == 0 ? eq : 0), warp_tot);
+    // block_scan2 is inclusive over threads; lane 0's value is the warp's inclusive total
+    const int gt_incl = __shfl_sync(0xffffffffu, inc.x, 0), eq_incl = __shfl_sync(0xffffffffu, inc.y, 0);
+    int eq_before = eq_incl - eq;
+    int pos = (gt_incl - gt) + min(eq_before, remaining);
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int64_t base = lo; base < hi; base += 32) {
+        const int64_t i = base + lane;
+        const uint32_t u = i < hi ? key_at(i) : 0u;
+        const bool is_eq = i < hi && u == T;
+        const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+        const int my_eq_rank = eq_before + __popc(eqm & lt_mask);
+        const bool take = i < hi && (u > T || (is_eq && my_eq_rank < remaining));
+        const unsigned tm = __ballot_sync(0xffffffffu, take);
+        if (take) {
+            const int p = pos + __popc(tm & lt_mask);
+            if (p < k) out[p] = int32_t(i);
+        }
+        pos += __popc(tm);
+        eq_before += __popc(eqm);
+    }
+}
+
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(
     const float* __restrict__ scores, int64_t ld, int64_t max_blocks,
     const int64_t* __restrict__ q_pos, int m, int W, int k, int32_t* __restrict__ idx) {
@@ -94,37 +138,120 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(
         __syncthreads();
     }
     // prefix is now the k-th largest key; `remaining` elements equal to it are taken.
-    const uint32_t T = prefix;
-    const int64_t seg = ceil_div(n, kTopkThreads);
-    const int64_t lo = min(n, tid * seg), hi = min(n, lo + seg);
-    int gt = 0, eq = 0;
-    for (int64_t i = lo; i < hi; ++i) {
-        const uint32_t u = order_key(s[i]);
-        gt += u > T;
-        eq += u == T;
+    write_selection_impl([&](int64_t i) { return order_key(s[i]); }, n, prefix, remaining, k, out, warp_tot);
+}
+
+// Rows that fit in shared memory: the row is read once into shared memory as
+// order keys; four passes of 8-bit digits find the k-th largest key.  Pass 0
+// sees every element: each warp counts into its own 256-bin histogram, and
+// lanes holding the same digit are merged with __match_any_sync so that one
+// leader adds their count (N(0, s) scores put most elements into a few
+// exponent bins, which would otherwise serialise the shared atomics).
+// Passes 1-3 only count the elements that still match the selected prefix.
+constexpr int kTopkSmemMax = 45056;  // keys kept in shared memory (176 KB)
+
+__global__ void __launch_bounds__(kTopkThreads) topk_smem_kernel(
+    const float* __restrict__ scores, int64_t ld, int64_t max_blocks,
+    const int64_t* __restrict__ q_pos, int m, int W, int k, int32_t* __restrict__ idx) {
+    extern __shared__ uint32_t keys[];                 // [n]
+    __shared__ int whist[32][256];
+    __shared__ int2 warp_tot[32];
+    __shared__ int found_digit, found_above;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int64_t row = blockIdx.x;
+    const float* s = scores + row * ld;
+    int32_t* out = idx + row * k;
+    const int n = int(min(n_elig(q_pos[row], m, W), max_blocks));
+    if (n <= k) {
+        for (int i = tid; i < k; i += kTopkThreads) out[i] = i < n ? i : -1;
+        return;
     }
-    const int2 inc = block_scan2(make_int2(gt, eq), warp_tot);
-    int eq_before = inc.y - eq;
-    int pos = (inc.x - gt) + min(eq_before, remaining);
-    for (int64_t i = lo; i < hi; ++i) {
-        const uint32_t u = order_key(s[i]);
-        if (u > T) {
-            if (pos < k) out[pos] = int32_t(i);
-            ++pos;
-        } else if (u == T) {
-            if (eq_before < remaining) {
-                if (pos < k) out[pos] = int32_t(i);
-                ++pos;
-            }
-            ++eq_before;
+    // fill: batches of 8 independent loads per thread so their latencies overlap
+    for (int base = 0; base < n; base += 8 * kTopkThreads) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = base + j * kTopkThreads + tid;
+            v[j] = i < n ? s[i] : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = base + j * kTopkThreads + tid;
+            if (i < n) keys[i] = order_key(v[j]);
         }
     }
+    for (int i = tid; i < 32 * 256; i += kTopkThreads) (&whist[0][0])[i] = 0;
+    __syncthreads();
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = k;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        if (pass == 0) {
+            for (int base = 0; base < n; base += kTopkThreads) {   // whole warps iterate together
+                const int i = base + tid;
+                const bool in = i < n;
+                const uint32_t dg = in ? (keys[i] >> 24) : 0xFFFFFFFFu;
+                const unsigned same = __match_any_sync(0xffffffffu, dg);
+                if (in && lane == __ffs(same) - 1) whist[wid][dg] += __popc(same);
+            }
+            __syncthreads();
+            if (tid < 256) {
+                int c = 0;
+                for (int w = 0; w < 32; ++w) c += whist[w][tid];
+                whist[0][tid] = c;
+            }
+        } else {
+            for (int i = tid; i < n; i += kTopkThreads) {
+                const uint32_t u = keys[i];
+                if ((u & pmask) == prefix) atomicAdd(&whist[0][(u >> shift) & 255], 1);
+            }
+        }
+        __syncthreads();
+        if (wid == 0) {
+            // lane l owns the 8 bins counted from the top: 255-8l .. 248-8l
+            int loc[8], sum = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { loc[j] = whist[0][255 - 8 * lane - j]; sum += loc[j]; }
+            int inc = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            int above = inc - sum;
+            if (above < remaining && remaining <= inc) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (above < remaining && remaining <= above + loc[j]) {
+                        found_digit = 255 - 8 * lane - j;
+                        found_above = above;
+                    }
+                    above += loc[j];
+                }
+            }
+        }
+        __syncthreads();
+        remaining -= found_above;
+        prefix |= uint32_t(found_digit) << shift;
+        pmask |= 0xFFu << shift;
+        if (tid < 256) whist[0][tid] = 0;
+        __syncthreads();
+    }
+    write_selection_impl([&](int64_t i) { return keys[i]; }, int64_t(n), prefix, remaining, k, out, warp_tot);
 }
 
 cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, const int64_t* q_pos,
                         int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
-    topk_kernel<<<unsigned(rows), kTopkThreads, 0, s>>>(scores, ld, max_blocks, q_pos, m, W, k, idx);
+    if (max_blocks <= kTopkSmemMax) {
+        const size_t sm = size_t(std::max<int64_t>(max_blocks, 1)) * 4;
+        cudaError_t e = ensure_smem(topk_smem_kernel, size_t(sm));
+        if (e != cudaSuccess) return e;
+        topk_smem_kernel<<<unsigned(rows), kTopkThreads, sm, s>>>(scores, ld, max_blocks, q_pos, m, W, k, idx);
+    } else {
+        topk_kernel<<<unsigned(rows), kTopkThreads, 0, s>>>(scores, ld, max_blocks, q_pos, m, W, k, idx);
+    }
     return cudaGetLastError();
 }
 

@@ -171,7 +171,7 @@ def test_indexer_matches_oracle(idx, HI, dI, n_q, nb, m, W):
 
 
 # --------------------------------------------------------------------- top-k
-@pytest.mark.parametrize("n,k", [(50, 8), (2015, 512), (32736, 512), (5000, 1024)])
+@pytest.mark.parametrize("n,k", [(50, 8), (2015, 512), (32736, 512), (5000, 1024), (60000, 1024)])
 def test_topk_matches_oracle_exactly(n, k):
     rows = 6
     s = synth.tensor_np(4, "ts", (rows, n))
