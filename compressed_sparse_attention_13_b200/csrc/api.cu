@@ -71,16 +71,18 @@ struct AttnPlan {
     size_t bytes() const { return n_splits > 1 ? part_o_bytes + part_ml_bytes : 0; }
 };
 
-// The tensor-core kernel runs one 217 KB CTA per SM, so its splits fill the
-// 148 SMs in a single wave with at least one 128-item tile per split.
+// The tensor-core kernel runs one ~215 KB CTA per SM, so its splits fill the
+// 148 SMs in a single wave with at least one 64-item tile per split.
 static int choose_splits_tc(int64_t rows, int64_t items_per_row) {
     if (rows >= kNumSMs) return 1;
-    const int64_t s = std::min<int64_t>(kNumSMs / rows, ceil_div(items_per_row, 128));
+    const int64_t s = std::min<int64_t>(kNumSMs / rows, ceil_div(items_per_row, 64));
     return int(std::max<int64_t>(1, std::min<int64_t>(s, 64)));
 }
 
 static AttnPlan plan_attn(const csa_params* p, int64_t rows, int64_t items_per_row) {
     AttnPlan a;
+    // (the tensor-core kernel is also limited to rows that fit 32 bits; with
+    // larger buffers the CUDA-core kernel runs with the same split count)
     a.n_splits = attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim)
                      ? choose_splits_tc(rows, items_per_row)
                      : choose_splits(rows, items_per_row);
@@ -111,7 +113,8 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
     a.n_q = n_q; a.n_splits = plan.n_splits; a.out = out;
     a.part_o = (float*)ws;
     a.part_ml = (float2*)((char*)ws + plan.part_o_bytes);
-    const bool tc = attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim);
+    const bool tc = attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim) &&
+                    attn_tc_rows_fit(max_entries, n_raw);
     int st = cuda_status(tc ? launch_attn_tc(a, rows, s) : launch_attn_simt(p->act_fmt, p->kv_fmt, a, rows, s));
     if (st) return st;
     if (plan.n_splits > 1)

@@ -186,33 +186,73 @@ static cudaError_t launch_attn_t(const AttnArgs& a, int64_t rows, cudaStream_t s
 }
 
 // Combine split partials: o = sum_s e^(m_s-M) O_s / (sum_s e^(m_s-M) l_s + e^(sink-M)).
+// One CTA per (row, head), 128 threads x 4 dims (D = 512; other widths loop).
+// The per-split weights are computed once into shared memory, then each
+// thread accumulates float4 slices with the split loads issued four at a time.
 template <int ACT>
 __global__ void __launch_bounds__(128) combine_kernel(int H, int D, int n_splits,
                                                       const float* __restrict__ part_o,
                                                       const float2* __restrict__ part_ml,
                                                       const float* __restrict__ sinks, void* out) {
+    __shared__ float wgt[64];
+    __shared__ float inv_s;
     const int64_t row = blockIdx.x;
     const int h = blockIdx.y;
     const float2* ml = part_ml + row * n_splits * H + h;
-    float M = sinks ? sinks[h] : -INFINITY;
-    for (int s = 0; s < n_splits; ++s) M = fmaxf(M, ml[s * H].x);
-    float den = sinks ? expf(sinks[h] - M) : 0.f;
-    if (M == -INFINITY) den = 0.f;
-    for (int s = 0; s < n_splits; ++s) {
-        const float2 v = ml[s * H];
-        if (v.x != -INFINITY) den += v.y * expf(v.x - M);
-    }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    for (int c = threadIdx.x; c < D; c += blockDim.x) {
-        float acc = 0.f;
-        for (int s = 0; s < n_splits; ++s) {
+    if (threadIdx.x < 32) {
+        float M = sinks ? sinks[h] : -INFINITY;
+        for (int s = threadIdx.x; s < n_splits; s += 32) M = fmaxf(M, ml[s * H].x);
+        M = warp_max(M);
+        float den = 0.f;
+        for (int s = threadIdx.x; s < n_splits; s += 32) {
             const float2 v = ml[s * H];
-            if (v.x == -INFINITY) continue;
-            acc = fmaf(expf(v.x - M), part_o[((row * n_splits + s) * H + h) * int64_t(D) + c], acc);
+            const float w = v.x == -INFINITY ? 0.f : expf(v.x - M);
+            wgt[s] = w;
+            den += w * v.y;
+        }
+        den = warp_sum(den);
+        if (threadIdx.x == 0) {
+            if (sinks && M != -INFINITY) den += expf(sinks[h] - M);
+            inv_s = den > 0.f ? 1.f / den : 0.f;
+        }
+    }
+    __syncthreads();
+    const float inv = inv_s;
+    const int64_t stride = int64_t(H) * D;  // between splits
+    for (int c = 4 * threadIdx.x; c < D; c += 4 * blockDim.x) {
+        const float* base = part_o + (row * n_splits * H + h) * int64_t(D) + c;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        int s = 0;
+        for (; s + 4 <= n_splits; s += 4) {
+            float4 v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const float4*>(base + (s + j) * stride);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float w = wgt[s + j];
+                if (w == 0.f) continue;  // an empty split adds nothing (its partial is not read)
+                acc.x = fmaf(w, v[j].x, acc.x); acc.y = fmaf(w, v[j].y, acc.y);
+                acc.z = fmaf(w, v[j].z, acc.z); acc.w = fmaf(w, v[j].w, acc.w);
+            }
+        }
+        for (; s < n_splits; ++s) {
+            const float w = wgt[s];
+            if (w == 0.f) continue;
+            const float4 v = *reinterpret_cast<const float4*>(base + s * stride);
+            acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
         }
         const int64_t o = (row * H + h) * int64_t(D) + c;
-        if constexpr (ACT == CSA_F32) ((float*)out)[o] = acc * inv;
-        else ((__nv_bfloat16*)out)[o] = __float2bfloat16_rn(acc * inv);
+        if constexpr (ACT == CSA_F32) {
+            *reinterpret_cast<float4*>((float*)out + o) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        } else {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t*>(&lo);
+            pk.y = *reinterpret_cast<uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>((__nv_bfloat16*)out + o) = pk;
+        }
     }
 }
 

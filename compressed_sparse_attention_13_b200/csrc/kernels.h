@@ -43,6 +43,7 @@ cudaError_t launch_indexer_tc(const void* qI, const void* qI_s, const float* w, 
 cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, const int64_t* q_pos,
                         int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s);
 bool attn_tc_supported(int act, int kvf, int H, int D);
+bool attn_tc_rows_fit(int64_t max_entries, int64_t n_raw);
 cudaError_t launch_attn_tc(const AttnArgs& a, int64_t rows, cudaStream_t s);
 cudaError_t launch_attn_simt(int act, int kvf, const AttnArgs& a, int64_t rows, cudaStream_t s);
 bool attn_simt_supported(int act, int kvf, int H, int D);
