@@ -8,7 +8,9 @@ anything without the built library raises.
 
 Names follow the C ABI: ``csa_compress``, ``csa_quantize``, ``indexer_score``,
 ``topk_select``, ``sparse_mqa_attn``, ``hca_attn``, ``csa_decode``,
-``csa_prefill``, ``csa_workspace_size``, ``csa_device_status``.
+``csa_prefill``, ``csa_workspace_size``, ``csa_device_status``, and
+``csa_decode_noalloc`` (csa_decode on the library's fixed device scratch, for
+callers that cannot allocate).
 """
 from __future__ import annotations
 
@@ -19,6 +21,8 @@ from dataclasses import dataclass
 F32, BF16, FP8_S64, MXFP4 = 0, 1, 2, 3
 OP_SPARSE_ATTN, OP_HCA_ATTN, OP_DECODE, OP_PREFILL = 0, 1, 2, 3
 DEV_BAD_INDEX, DEV_RANGE, DEV_TIMEOUT = 0x1, 0x2, 0x4
+NOALLOC_SCRATCH_BYTES = 32 << 20   # CSA_NOALLOC_SCRATCH_BYTES
+ERR_WORKSPACE = -4
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libcsa13.so")
@@ -47,7 +51,7 @@ def params(m, window, top_k, n_heads, head_dim, idx_heads, idx_dim, scale,
 
 EXPORTS = ["csa_compress", "csa_quantize", "indexer_score", "topk_select", "sparse_mqa_attn",
            "hca_attn", "csa_decode", "csa_prefill", "csa_workspace_size", "csa_device_status",
-           "csa_strerror", "csa_version"]
+           "csa_strerror", "csa_version", "csa_decode_noalloc"]
 
 
 def lib():
@@ -70,6 +74,8 @@ def lib():
                                  C.c_size_t, P]
         L.csa_prefill.argtypes = [PP, I32, I64, I64, P, I64, I64, P, P, P, P, P, P, P, P, P, P,
                                   I64, P, P, P, P, C.c_size_t, P]
+        L.csa_decode_noalloc.argtypes = [PP, I32, P, P, P, P, P, P, P, P, I64, P, I64, P, P, P,
+                                         P, P, P]
         L.csa_workspace_size.restype = C.c_size_t
         L.csa_workspace_size.argtypes = [PP, I32, I32, I64, I64]
         L.csa_device_status.argtypes = [P, C.POINTER(C.c_uint32), I32]
@@ -189,6 +195,18 @@ def csa_decode(p: Params, batch: int, q, qI: Stored, w, kv: Stored, kI: Stored, 
         C.byref(p), batch, _p(q), _p(qI.data), _p(qI.scales), _p(w), _p(kv.data), _p(kv.scales),
         _p(kI.data), _p(kI.scales), max_blocks, _p(raw), n_raw, _p(raw_pos0), _p(q_pos),
         _p(sinks), _p(out), _p(idx_out), wp, wb, _s(stream)))
+
+
+def csa_decode_noalloc(p: Params, batch: int, q, qI: Stored, w, kv: Stored, kI: Stored,
+                       max_blocks: int, raw, n_raw: int, raw_pos0, q_pos, sinks, out, idx_out,
+                       stream=None):
+    """csa_decode without a workspace argument: the library's fixed device scratch
+    is used instead.  Calls on one device must not overlap; requests larger than
+    NOALLOC_SCRATCH_BYTES raise CsaError with status ERR_WORKSPACE."""
+    _ok("csa_decode_noalloc", lib().csa_decode_noalloc(
+        C.byref(p), batch, _p(q), _p(qI.data), _p(qI.scales), _p(w), _p(kv.data), _p(kv.scales),
+        _p(kI.data), _p(kI.scales), max_blocks, _p(raw), n_raw, _p(raw_pos0), _p(q_pos),
+        _p(sinks), _p(out), _p(idx_out), _s(stream)))
 
 
 def csa_prefill(p: Params, batch: int, T: int, t0: int, raw, n_raw: int, raw_pos0: int, z, bias,

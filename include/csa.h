@@ -223,6 +223,52 @@ int csa_prefill(const csa_params* p, int32_t batch, int64_t T, int64_t t0, const
 size_t csa_workspace_size(const csa_params* p, int32_t op, int32_t batch, int64_t n_q,
                           int64_t n_ctx);
 
+/* ------------------------------------------------------------------------
+ * csa_decode_noalloc -- csa_decode for callers that cannot allocate device
+ * memory.  The method itself has no counterpart of this call: it exists
+ * only to serve such callers, because csa_decode needs a workspace.  Examples
+ * are a host program with no device allocator of its own, a decode loop
+ * that must not call cudaMalloc between steps (cudaMalloc synchronises the
+ * device), and a server whose device memory is all committed at start-up.
+ *
+ * It computes exactly what csa_decode computes, with the same kernels and
+ * the same arguments, minus `workspace` and `ws_bytes`.  The scores,
+ * selection and split-K partials go to a fixed scratch area that the library
+ * reserves statically on each device: CSA_NOALLOC_SCRATCH_BYTES, which is
+ * 32 MiB.  At m = 4, k = 512, W = 128 and 64 heads of 512, that covers any
+ * batch of 1 to 252 sequences of 128K tokens, or 32 sequences of up to
+ * 500,000 tokens.  Nothing is allocated, not even on the first call.
+ *
+ *   errors: CSA_ERR_WORKSPACE, with nothing launched, when
+ *           csa_workspace_size(p, CSA_OP_DECODE, batch, 1, max_blocks) is
+ *           larger than CSA_NOALLOC_SCRATCH_BYTES.  Otherwise the errors are
+ *           those of csa_decode.  CSA_ERR_CUDA if the scratch address cannot
+ *           be found on the current device.
+ *   device: the scratch belongs to the device that is current on the
+ *           calling thread.  The stream and all pointers must belong to
+ *           that device too.
+ *   first call: on each device, the first call looks up the scratch's
+ *           address.  That lookup may load the library's device code.  So
+ *           make the first call on each device outside any stream capture,
+ *           before the calls you intend to record.
+ *   initial contents: none required.  Each scratch byte a call reads was
+ *           written earlier in the same call, so nothing needs to start at
+ *           zero.  The device status word (csa_device_status) is separate
+ *           from the scratch and behaves as for csa_decode.
+ *   overlap: every call on a device shares the one scratch area.  Two calls
+ *           on that device whose work can overlap race on it and corrupt
+ *           each other's results: calls from different streams, or from
+ *           different host threads.  Order them on one stream or with events.
+ * ------------------------------------------------------------------------ */
+#define CSA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+int csa_decode_noalloc(const csa_params* p, int32_t batch, const void* q, const void* qI,
+                       const void* qI_scales, const float* w, const void* kv,
+                       const void* kv_scales, const void* kI, const void* kI_scales,
+                       int64_t max_blocks, const void* raw, int64_t n_raw,
+                       const int64_t* raw_pos0, const int64_t* q_pos, const float* sinks,
+                       void* out, int32_t* idx_out, csa_stream_t stream);
+
 /* Synchronise `stream`, return the device status word (CSA_DEV_* bits) in
  * *flags, and clear it if `reset` is non-zero.  The word is shared by every
  * call on the current device. */
