@@ -17,14 +17,21 @@
 // TMEM lane j owns key j's 64 head scores and reduces them without any
 // cross-thread traffic.
 //
-// Persistent CTAs take contiguous ranges of (query row, 128-key tile) units.
-// Warp roles:
+// Persistent CTAs take contiguous ranges of (query row, 128-key tile) units
+// and walk them in order, skipping tiles past the row's eligible blocks; the
+// k-th eligible tile of a CTA is "tile it = k".  Warp roles:
 //   warp 0      bulk-async copies of raw key tiles (packed E2M1 + E8M0) into a
 //               kRawStages ring (one elected lane), TMEM allocation
 //   warp 1      MMA issue (one elected lane)
-//   warps 2-5   convert a raw tile to the E4M3 A tile; convert the query block
-//               to the E4M3 B tile when the row changes
-//   warps 6-9   epilogue: TMEM -> ReLU, weight, sum over heads -> score
+//   warps 2-9   two converter groups of four warps; group g converts the tiles
+//               with it % 2 == g into A buffer it % 4, and the query block of
+//               a row into query buffer (row count % 4) when its tile is the
+//               first of that row
+//   warps 10-17 two epilogue groups; group g reads accumulator it % 4 of its
+//               tiles from TMEM, applies ReLU, weights and sums over heads
+// Query buffers are safe to overwrite: the converter of tile it waits for the
+// MMA of tile it - 4 (its A buffer), and MMAs complete in issue order; four
+// row changes need at least four tiles.
 // All waits are bounded (sm100::mbar_wait); after a timed-out wait a role
 // keeps iterating without waiting or touching memory, so every thread still
 // reaches the named and final barriers.
@@ -37,13 +44,16 @@ namespace {
 
 constexpr int kHI = 64, kDI = 128;
 constexpr int kTileKeys = 128;
-constexpr int kRawStages = 12;
+constexpr int kRawStages = 10;
+constexpr int kABufs = 4, kAccBufs = 4, kQBufs = 4;
+constexpr int kAccCols = 64;
 constexpr int kKeyBytes = kDI / 2;                           // 64
 constexpr int kRawData = kTileKeys * kKeyBytes;              // 8192
 constexpr int kRawBytes = kRawData + kTileKeys * (kDI / 32); // + 512 scale bytes
 constexpr int kATile = kTileKeys * kDI;                      // 16384 (E4M3)
 constexpr int kQTile = kHI * kDI;                            // 8192
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
+constexpr int kConvWarp0 = 2, kEpiWarp0 = 10;
 constexpr int kLutMinX = -8, kLutMaxX = 6;  // exponents whose E2M1 x 2^X are all E4M3 values
 
 struct IdxTcArgs {
@@ -60,20 +70,45 @@ struct IdxTcArgs {
 };
 
 struct Smem {
-    uint8_t a[2][kATile];              // 1024-aligned: E4M3 A tiles
-    uint8_t q[2][kQTile];              // E4M3 B tiles (query blocks)
+    uint8_t a[kABufs][kATile];         // 1024-aligned: E4M3 A tiles
+    uint8_t q[kQBufs][kQTile];         // E4M3 B tiles (query blocks)
     uint8_t raw[kRawStages][kRawBytes];
-    float ew[kHI];                     // epilogue-private weights of the current row
+    float ew[2][kHI];                  // per epilogue group: weights of its current row
     uint2 lut[kLutMaxX - kLutMinX + 1];  // E2M1 x 2^X -> E4M3 byte tables
     uint64_t raw_full[kRawStages], raw_empty[kRawStages];
-    uint64_t a_full[2], a_empty[2], acc_full[2], acc_empty[2];
+    uint64_t a_full[kABufs], a_empty[kABufs], acc_full[kAccBufs], acc_empty[kAccBufs];
     uint32_t tmem_base;
-    int abort_flag;
 };
 
-__device__ __forceinline__ int64_t unit_elig(const IdxTcArgs& a, int64_t row) {
-    return min(n_elig(a.q_pos[row], a.m, a.W), a.max_blocks);
-}
+// In-order walk over a CTA's units that visits only eligible tiles.  Rows
+// change at most once per tile; q_pos is read once per row.
+struct TileWalk {
+    int64_t u, u1, row, tile, ne, tpr;
+    bool started;
+    __device__ __forceinline__ TileWalk(const IdxTcArgs& a, int64_t u0, int64_t u_end)
+        : u(u0), u1(u_end), tpr(a.tiles_per_row), started(false) {
+        row = u0 / tpr;
+        tile = u0 - row * tpr;
+        ne = u0 < u_end ? min(n_elig(a.q_pos[row], a.m, a.W), a.max_blocks) : 0;
+    }
+    // Advance to the next eligible tile; false when the range is exhausted.
+    __device__ __forceinline__ bool next(const IdxTcArgs& a) {
+        if (started) { ++u; ++tile; }
+        started = true;
+        while (u < u1) {
+            if (tile == tpr) {
+                tile = 0;
+                ++row;
+                ne = min(n_elig(a.q_pos[row], a.m, a.W), a.max_blocks);
+            }
+            if (tile * kTileKeys < ne) return true;
+            u += tpr - tile;  // rest of this row is ineligible
+            tile = tpr;
+        }
+        return false;
+    }
+    __device__ __forceinline__ int64_t k0() const { return tile * kTileKeys; }
+};
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t d;
@@ -110,6 +145,19 @@ __device__ __forceinline__ uint2 e2m1x8_to_e4m3x8(uint32_t w, uint2 lut) {
 }
 
 
+__device__ __forceinline__ uint64_t pack_f32x2(float x, float y) {
+    return uint64_t(__float_as_uint(x)) | (uint64_t(__float_as_uint(y)) << 32);
+}
+__device__ __forceinline__ float2 unpack_f32x2(uint64_t v) {
+    return make_float2(__uint_as_float(uint32_t(v)), __uint_as_float(uint32_t(v >> 32)));
+}
+// (a.x*b.x + c.x, a.y*b.y + c.y), each rounded once
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 // Table entry for an E8M0 byte; flags exponents outside the exact range.
 __device__ __forceinline__ uint2 lut_for(const uint2* table, uint32_t e8m0) {
     int X = int(e8m0) - 127;
@@ -130,14 +178,11 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const IdxTcArgs
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRawStages; ++i) { mbar_init(&S.raw_full[i], 1); mbar_init(&S.raw_empty[i], 128); }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.a_full[i], 128); mbar_init(&S.a_empty[i], 1);
-            mbar_init(&S.acc_full[i], 1); mbar_init(&S.acc_empty[i], 128);
-        }
-        S.abort_flag = 0;
+        for (int i = 0; i < kABufs; ++i) { mbar_init(&S.a_full[i], 128); mbar_init(&S.a_empty[i], 1); }
+        for (int i = 0; i < kAccBufs; ++i) { mbar_init(&S.acc_full[i], 1); mbar_init(&S.acc_empty[i], 128); }
         fence_mbar_init();
     }
-    if (warp == 0) { tmem_alloc(&S.tmem_base, 128); tmem_relinquish(); }
+    if (warp == 0) { tmem_alloc(&S.tmem_base, kAccBufs * kAccCols); tmem_relinquish(); }
     if (threadIdx.x >= 64 && threadIdx.x < 64 + (kLutMaxX - kLutMinX + 1))
         S.lut[threadIdx.x - 64] = make_e4m3_lut(int(threadIdx.x) - 64 + kLutMinX);
     tc_fence_before();
@@ -151,71 +196,77 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const IdxTcArgs
     if (warp == 0) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
-            int64_t it = 0;
+            TileWalk tw(a, u0, u1);
+            int st = 0, issued = 0;
+            uint32_t ph = 0;
             bool ok = true;
-            for (int64_t u = u0; u < u1 && ok; ++u) {
-                const int64_t row = u / a.tiles_per_row, tile = u % a.tiles_per_row;
-                const int64_t ne = unit_elig(a, row);
-                const int64_t k0 = tile * kTileKeys;
-                if (k0 >= ne) continue;
-                const int st = int(it % kRawStages);
-                if (it >= kRawStages) ok = mbar_wait(&S.raw_empty[st], uint32_t((it / kRawStages - 1) & 1));
+            for (int it = 0; ok && tw.next(a); ++it) {
+                if (it >= kRawStages) ok = mbar_wait(&S.raw_empty[st], ph ^ 1u);
                 if (!ok) break;
-                int64_t nk = min(int64_t(kTileKeys), ne - k0);
+                ++issued;
+                const int64_t k0 = tw.k0();
+                int64_t nk = min(int64_t(kTileKeys), tw.ne - k0);
                 nk = min((nk + 3) & ~int64_t(3), a.max_blocks - k0);  // max_blocks % 4 == 0
-                const int64_t b = row / a.n_q;
-                const int64_t key0 = b * a.max_blocks + k0;
+                const int64_t key0 = (tw.row / a.n_q) * a.max_blocks + k0;
                 mbar_arrive_expect_tx(&S.raw_full[st], uint32_t(nk * (kKeyBytes + 4)));
                 bulk_g2s(S.raw[st], a.kI + key0 * kKeyBytes, uint32_t(nk * kKeyBytes), &S.raw_full[st]);
                 bulk_g2s(S.raw[st] + kRawData, a.kIs + key0 * 4, uint32_t(nk * 4), &S.raw_full[st]);
-                ++it;
+                if (++st == kRawStages) { st = 0; ph ^= 1u; }
             }
+            // Let every copy still in flight land before the CTA exits (already
+            // the case unless a consumer gave up on a wait).
+            for (int i = max(0, issued - kRawStages); i < issued; ++i)
+                if (!mbar_wait(&S.raw_full[i % kRawStages], uint32_t(i / kRawStages) & 1u)) break;
         }
     } else if (warp == 1) {
         // --------------------------------------------------------------- MMA
         if (lane == 0) {
             const uint32_t idesc = instr_desc(0, 0, 0, 0, 128, 64);  // E4M3 x E4M3, K-major
-            int64_t it = 0, cur_row = -1;
-            int qbuf = 1;
+            TileWalk tw(a, u0, u1);
+            int64_t cur_row = -1;
+            int rc = -1;
             bool ok = true;
-            for (int64_t u = u0; u < u1 && ok; ++u) {
-                const int64_t row = u / a.tiles_per_row, tile = u % a.tiles_per_row;
-                if (tile * kTileKeys >= unit_elig(a, row)) continue;
-                if (row != cur_row) { cur_row = row; qbuf ^= 1; }
-                const int s = int(it & 1);
-                ok = mbar_wait(&S.a_full[s], uint32_t((it >> 1) & 1));
-                if (ok && it >= 2) ok = mbar_wait(&S.acc_empty[s], uint32_t(((it >> 1) - 1) & 1));
+            for (int it = 0; ok && tw.next(a); ++it) {
+                if (tw.row != cur_row) { cur_row = tw.row; ++rc; }
+                const int b = it & (kABufs - 1);
+                const uint32_t par = uint32_t(it >> 2) & 1u;
+                ok = mbar_wait(&S.a_full[b], par);
+                if (ok && it >= kAccBufs) ok = mbar_wait(&S.acc_empty[b], par ^ 1u);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(S.a[s]), b0 = smem_u32(S.q[qbuf]);
+                const uint32_t a0 = smem_u32(S.a[b]), b0 = smem_u32(S.q[rc & (kQBufs - 1)]);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_f8(tmem + s * 64, smem_desc(a0 + k * 32, 16, 1024), smem_desc(b0 + k * 32, 16, 1024),
-                           idesc, k > 0);
-                mma_commit(&S.a_empty[s]);
-                mma_commit(&S.acc_full[s]);
-                ++it;
+                    mma_f8(tmem + b * kAccCols, smem_desc(a0 + k * 32, 16, 1024),
+                           smem_desc(b0 + k * 32, 16, 1024), idesc, k > 0);
+                mma_commit(&S.a_empty[b]);
+                mma_commit(&S.acc_full[b]);
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < kEpiWarp0) {
         // --------------------------------------------------------- converters
-        const int t = threadIdx.x - 64;  // 0..127
-        int64_t it = 0, cur_row = -1;
-        int qbuf = 1;
+        const int g = (warp - kConvWarp0) >> 2;         // group: tiles with it % 2 == g
+        const int t = threadIdx.x - 32 * (kConvWarp0 + 4 * g);  // 0..127
+        TileWalk tw(a, u0, u1);
+        int64_t cur_row = -1;
+        int rc = -1, rs = 0;
+        uint32_t rph = 0;
         bool ok = true;
-        for (int64_t u = u0; u < u1 && ok; ++u) {
-            const int64_t row = u / a.tiles_per_row, tile = u % a.tiles_per_row;
-            const int64_t ne = unit_elig(a, row);
-            const int64_t k0 = tile * kTileKeys;
-            if (k0 >= ne) continue;
-            const int s = int(it & 1);
-            if (it >= 2) ok = mbar_wait(&S.a_empty[s], uint32_t(((it >> 1) - 1) & 1));
+        for (int it = 0; ok && tw.next(a); ++it) {
+            const bool first_of_row = tw.row != cur_row;
+            if (first_of_row) { cur_row = tw.row; ++rc; }
+            const int my_rs = rs;
+            const uint32_t my_rph = rph;
+            if (++rs == kRawStages) { rs = 0; rph ^= 1u; }
+            if ((it & 1) != g) continue;
+            const int b = it & (kABufs - 1);
+            if (it >= kABufs) ok = mbar_wait(&S.a_empty[b], (uint32_t(it >> 2) & 1u) ^ 1u);
             if (!ok) break;
-            if (row != cur_row) {
+            if (first_of_row) {
                 // query block of this row -> E4M3 B tile: thread t does head t/2, half t%2
-                cur_row = row;
-                qbuf ^= 1;
                 const int h = t >> 1, half = t & 1;
+                const int64_t row = tw.row;
+                uint8_t* qdst = S.q[rc & (kQBufs - 1)];
                 const uint8_t* src = a.qI + (row * kHI + h) * kKeyBytes + half * 32;
                 const uint8_t* srs = a.qIs + (row * kHI + h) * 4 + half * 2;
                 const uint4 p0 = *reinterpret_cast<const uint4*>(src);
@@ -227,82 +278,88 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const IdxTcArgs
                     const uint2 sc = c < 2 ? s0 : s1;
                     const uint2 lo = e2m1x8_to_e4m3x8(pw[2 * c], sc);
                     const uint2 hi = e2m1x8_to_e4m3x8(pw[2 * c + 1], sc);
-                    *reinterpret_cast<uint4*>(S.q[qbuf] + sw128_offset(h, half * 4 + c)) =
+                    *reinterpret_cast<uint4*>(qdst + sw128_offset(h, half * 4 + c)) =
                         make_uint4(lo.x, lo.y, hi.x, hi.y);
                 }
             }
-            const int rs = int(it % kRawStages);
-            ok = mbar_wait(&S.raw_full[rs], uint32_t((it / kRawStages) & 1));
+            ok = mbar_wait(&S.raw_full[my_rs], my_rph);
             if (!ok) break;
             // four consecutive threads share a key, one 32-element MX block each:
             // 16-byte reads at consecutive addresses, two swizzled 16-byte writes
+            const int64_t k0 = tw.k0(), ne = tw.ne;
             const int blk = t & 3;
+            const uint8_t* raw = S.raw[my_rs];
 #pragma unroll
             for (int pass = 0; pass < 4; ++pass) {
                 const int key = (t >> 2) + 32 * pass;
                 uint4 o0 = make_uint4(0, 0, 0, 0), o1 = o0;
                 if (k0 + key < ne) {
-                    const uint4 pk = *reinterpret_cast<const uint4*>(S.raw[rs] + key * kKeyBytes + 16 * blk);
-                    const uint2 sc = lut_for(S.lut, S.raw[rs][kRawData + key * 4 + blk]);
+                    const uint4 pk = *reinterpret_cast<const uint4*>(raw + key * kKeyBytes + 16 * blk);
+                    const uint2 sc = lut_for(S.lut, raw[kRawData + key * 4 + blk]);
                     const uint2 e0 = e2m1x8_to_e4m3x8(pk.x, sc), e1 = e2m1x8_to_e4m3x8(pk.y, sc);
                     const uint2 e2 = e2m1x8_to_e4m3x8(pk.z, sc), e3 = e2m1x8_to_e4m3x8(pk.w, sc);
                     o0 = make_uint4(e0.x, e0.y, e1.x, e1.y);
                     o1 = make_uint4(e2.x, e2.y, e3.x, e3.y);
                 }
-                *reinterpret_cast<uint4*>(S.a[s] + sw128_offset(key, 2 * blk)) = o0;
-                *reinterpret_cast<uint4*>(S.a[s] + sw128_offset(key, 2 * blk + 1)) = o1;
+                *reinterpret_cast<uint4*>(S.a[b] + sw128_offset(key, 2 * blk)) = o0;
+                *reinterpret_cast<uint4*>(S.a[b] + sw128_offset(key, 2 * blk + 1)) = o1;
             }
             fence_proxy_async_smem();
-            mbar_arrive(&S.raw_empty[rs]);
-            mbar_arrive(&S.a_full[s]);
-            ++it;
+            mbar_arrive(&S.raw_empty[my_rs]);
+            mbar_arrive(&S.a_full[b]);
         }
     } else {
         // ----------------------------------------------------------- epilogue
+        const int g = (warp - kEpiWarp0) >> 2;        // group: tiles with it % 2 == g
         const int sub = warp & 3;                     // TMEM lane quarter of this warp
         const int key = sub * 32 + lane;              // key within the tile
-        const int et = threadIdx.x - 192;             // 0..127
-        int64_t it = 0, cur_row = -1;
+        const int et = threadIdx.x - 32 * (kEpiWarp0 + 4 * g);  // 0..127
+        float* ew = S.ew[g];
+        TileWalk tw(a, u0, u1);
+        int64_t cur_row = -1;
         bool ok = true;
-        for (int64_t u = u0; u < u1; ++u) {
-            const int64_t row = u / a.tiles_per_row, tile = u % a.tiles_per_row;
-            const int64_t ne = unit_elig(a, row);
-            const int64_t k0 = tile * kTileKeys;
-            if (k0 >= ne) continue;
-            if (row != cur_row) {  // every epilogue thread takes this branch together
-                cur_row = row;
-                named_bar(2, 128);
-                if (et < kHI) S.ew[et] = a.w[row * kHI + et];
-                named_bar(2, 128);
+        for (int it = 0; tw.next(a); ++it) {
+            if ((it & 1) != g) continue;
+            if (tw.row != cur_row) {  // every thread of the group takes this branch together
+                cur_row = tw.row;
+                named_bar(2 + g, 128);
+                if (et < kHI) ew[et] = a.w[cur_row * kHI + et];
+                named_bar(2 + g, 128);
             }
-            const int s = int(it & 1);
-            if (ok) ok = mbar_wait(&S.acc_full[s], uint32_t((it >> 1) & 1));
-            if (!ok) { ++it; continue; }
+            const int b = it & (kAccBufs - 1);
+            if (ok) ok = mbar_wait(&S.acc_full[b], uint32_t(it >> 2) & 1u);
+            if (!ok) continue;
             tc_fence_after();
-            float v[4][16];
-            const uint32_t base = tmem + (uint32_t(sub * 32) << 16) + s * 64;
+            const uint32_t base = tmem + (uint32_t(sub * 32) << 16) + b * kAccCols;
+            // two interleaved partial sums, packed fma over (even, odd) heads;
+            // the 64 head columns are read in two halves
+            uint64_t acc2 = 0;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld16(base + 16 * c, v[c]);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&S.acc_empty[s]);
-            float acc = 0.f;
+            for (int hf = 0; hf < 2; ++hf) {
+                float v[2][16];
+                tmem_ld16(base + 32 * hf, v[0]);
+                tmem_ld16(base + 32 * hf + 16, v[1]);
+                tmem_wait_ld();
+                if (hf == 1) {
+                    tc_fence_before();
+                    mbar_arrive(&S.acc_empty[b]);
+                }
 #pragma unroll
-            for (int h = 0; h < 64; h += 4) {
-                const float4 wv = *reinterpret_cast<const float4*>(&S.ew[h]);
-                acc = fmaf(wv.x, fmaxf(v[h >> 4][h & 15], 0.f), acc);
-                acc = fmaf(wv.y, fmaxf(v[h >> 4][(h & 15) + 1], 0.f), acc);
-                acc = fmaf(wv.z, fmaxf(v[h >> 4][(h & 15) + 2], 0.f), acc);
-                acc = fmaf(wv.w, fmaxf(v[h >> 4][(h & 15) + 3], 0.f), acc);
+                for (int h = 0; h < 32; h += 2) {
+                    const float2 wv = *reinterpret_cast<const float2*>(&ew[32 * hf + h]);
+                    const float r0 = fmaxf(v[h >> 4][h & 15], 0.f);
+                    const float r1 = fmaxf(v[h >> 4][(h & 15) + 1], 0.f);
+                    acc2 = fma_f32x2(pack_f32x2(wv.x, wv.y), pack_f32x2(r0, r1), acc2);
+                }
             }
-            const int64_t j = k0 + key;
-            if (j < ne) a.scores[row * a.ld + j] = acc;
-            ++it;
+            const float2 accs = unpack_f32x2(acc2);
+            const int64_t j = tw.k0() + key;
+            if (j < tw.ne) a.scores[cur_row * a.ld + j] = accs.x + accs.y;
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 128);
+    if (warp == 0) tmem_dealloc(tmem, kAccBufs * kAccCols);
 }
 
 bool indexer_tc_supported(int fmt, int HI, int dI, int64_t max_blocks) {
