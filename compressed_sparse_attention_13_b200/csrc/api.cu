@@ -193,7 +193,8 @@ int indexer_score(const csa_params* p, int32_t batch, int32_t n_q, const void* q
     if (!aligned16(qI) || !aligned16(kI) || !aligned16(scores) || !aligned16(qI_scales) ||
         !aligned16(kI_scales))
         return CSA_ERR_ALIGN;
-    if (indexer_tc_supported(p->idx_fmt, p->idx_heads, p->idx_dim, max_blocks))
+    if (indexer_tc_supported(p->idx_fmt, p->idx_heads, p->idx_dim, max_blocks, batch,
+                             int64_t(batch) * n_q))
         return cuda_status(launch_indexer_tc(qI, qI_scales, w, kI, kI_scales, max_blocks, q_pos,
                                              batch, n_q, p->m, p->window, scores, ld_scores,
                                              (cudaStream_t)stream));

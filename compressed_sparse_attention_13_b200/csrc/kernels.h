@@ -35,7 +35,7 @@ cudaError_t launch_indexer_simt(int fmt, int HI, int dI, int m, int W, const voi
                                 const void* kI_s, int64_t max_blocks, const int64_t* q_pos,
                                 int batch, int n_q, int64_t max_elig, float* scores, int64_t ld,
                                 cudaStream_t s);
-bool indexer_tc_supported(int fmt, int HI, int dI, int64_t max_blocks);
+bool indexer_tc_supported(int fmt, int HI, int dI, int64_t max_blocks, int64_t batch, int64_t rows);
 cudaError_t launch_indexer_tc(const void* qI, const void* qI_s, const float* w, const void* kI,
                               const void* kI_s, int64_t max_blocks, const int64_t* q_pos,
                               int batch, int n_q, int m, int W, float* scores, int64_t ld,

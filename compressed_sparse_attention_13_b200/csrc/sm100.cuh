@@ -90,6 +90,18 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// 2-D tiled tensor copy global -> shared (no multicast), completing the box's
+// bytes on bar.  `map` is a __grid_constant__ kernel parameter; x is the
+// innermost coordinate and must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(void* dst_smem, const void* map, int32_t x, int32_t y,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst_smem)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // ------------------------------------------------------------------ TMEM
 // Allocate `ncols` (power of two >= 32) TMEM columns; the base address is
 // written to *dst_smem.  Executed by one full warp.
@@ -185,6 +197,22 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
         : "memory");
 }
 
+// 32 lanes x 32 bits, 4 / 8 consecutive columns: thread i of the warp writes
+// row (lane base + i).
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c,
+                                         uint32_t d) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(a),
+                 "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                     taddr),
+                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                 "r"(v[7])
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -235,6 +263,27 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_
         : "memory");
 }
 
+// Block-scaled MMA on packed E2M1 operands (kind::mxf4, one E8M0 scale per 32
+// elements along K, K = 64 per instruction).  sfa / sfb are the TMEM addresses
+// of the scale factors: row r of A (of B) finds its two scales in bytes 0 and
+// 1 of lane r % 32, column r / 32 past the address, replicated in all four
+// lane quarters.
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// Instruction descriptor for kind::mxf4 with E8M0 scales: A and B E2M1,
+// K-major, N >> 3 and M >> 4 (the accumulator is fp32).
+__host__ __device__ constexpr uint32_t instr_desc_mxf4(uint32_t M, uint32_t N) {
+    return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24);
+}
+
 // Arrive once on `bar` when every MMA issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile(
@@ -248,6 +297,13 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 // 1024 bytes apart (the canonical K-major SW128 layout).
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
     return (row >> 3) * 1024u + (row & 7u) * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..3) of row `row` inside a
+// 64-byte-swizzled tile of 64-byte rows (8-row groups 512 bytes apart), the
+// layout a 2-D tensor copy with 64-byte swizzle writes.
+__device__ __forceinline__ uint32_t sw64_offset(uint32_t row, uint32_t chunk) {
+    return row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
 }
 
 // Named barrier among `count` threads (a multiple of 32).

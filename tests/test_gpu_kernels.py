@@ -278,17 +278,36 @@ def test_out_of_range_index_is_flagged_not_read():
     assert torch.isfinite(out).all()
 
 
-def test_mxfp4_scale_outside_exact_range_is_flagged():
-    """The tensor-core indexer converts E2M1 x 2^X to E4M3 exactly only for X
-    in [-8, 6]; a larger block exponent must raise CSA_DEV_RANGE."""
-    HI, dI, nb, m, W = 64, 128, 256, 4, 128
-    qv = synth.tensor_np(8, "rq", (1, 1, HI, dI))
-    kv_ = synth.tensor_np(8, "rk", (1, nb, dI)) * 1e4      # X around 11
-    w = synth.tensor_np(8, "rw", (1, 1, HI), std=0.1)
-    q_pos = np.array([[m * nb + W]], np.int64)
+def test_mxfp4_indexer_exact_across_block_exponents():
+    """The block-scaled tensor-core indexer applies E8M0 exponents in the MMA
+    itself, so keys and queries whose blocks span a wide exponent range (per
+    key 2^-40 .. 2^40, per block a further 2^+-10, per query head 2^+-20) still
+    match the oracle within the fp32 accumulation bound, and nothing is flagged."""
+    HI, dI, nb, m, W, batch, n_q = 64, 128, 640, 4, 128, 2, 2
+    rng = np.random.default_rng(81)
+    qv = synth.tensor_np(8, "rq", (batch, n_q, HI, dI))
+    qv = qv * np.exp2(rng.integers(-20, 21, (batch, n_q, HI, 1)))
+    kv_ = synth.tensor_np(8, "rk", (batch, nb, dI))
+    kv_ = kv_ * np.exp2(rng.integers(-40, 41, (batch, nb, 1)))
+    kv_ = kv_ * np.repeat(np.exp2(rng.integers(-10, 11, (batch, nb, dI // 32))), 32, axis=2)
+    w = synth.tensor_np(8, "rw", (batch, n_q, HI), std=0.1)
+    q_pos = np.array([[m * nb + W, m * 300 + W + 3], [m * nb + W + 7, m * 129 + W]], np.int64)
     p = K.params(m, W, 16, 1, 64, HI, dI, 1.0, idx_fmt=K.MXFP4)
-    qd, _ = both_stored(qv.reshape(-1, dI), "mxfp4")
-    kd, _ = both_stored(kv_.reshape(-1, dI), "mxfp4")
-    scores = torch.zeros((1, 1, nb), device="cuda")
-    K.indexer_score(p, 1, 1, qd, up(w), kd, nb, up(q_pos), scores, nb)
-    assert K.csa_device_status(reset=True) & K.DEV_RANGE
+    qd, _ = both_stored(qv.reshape(-1, dI).astype(np.float32), "mxfp4")
+    kd, _ = both_stored(kv_.reshape(-1, dI).astype(np.float32), "mxfp4")
+    scores = torch.full((batch, n_q, nb), float("nan"), device="cuda")
+    K.indexer_score(p, batch, n_q, qd, up(w), kd, nb, up(q_pos), scores, nb)
+    assert K.csa_device_status(reset=True) == 0
+    got = down(scores)
+    for b in range(batch):
+        qo = orc_quantize(qv[b].reshape(-1, dI).astype(np.float32), "mxfp4")
+        ko = orc_quantize(kv_[b].astype(np.float32), "mxfp4")
+        ref = oracle.indexer(qo, w[b], ko, q_pos[b], HI, m, W)
+        qdq = oracle.dequantize(qo).reshape(n_q, HI, dI)
+        kdq = oracle.dequantize(ko)
+        for i in range(n_q):
+            ne = min(oracle.n_elig(int(q_pos[b, i]), m, W), nb)
+            mag = (np.abs(w[b, i])[:, None] * np.linalg.norm(qdq[i], axis=1)[:, None] *
+                   np.linalg.norm(kdq[:ne], axis=1)[None, :]).sum(0)
+            err = np.abs(got[b, i, :ne] - ref[i, :ne])
+            assert (err <= 1e-5 * mag + 1e-30).all(), (b, i, err.max())
