@@ -143,6 +143,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) 
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
     const uint32_t tS = tmem, tO = tmem + 128;  // S[buf]: cols [64 buf, 64 buf + 64); O^T quarter q: [128+64q, 192+64q)
+    const uint8_t* kv_seq = (const uint8_t*)a.kv + b * a.max_entries * int64_t(kD);
+    const float* kvs_seq = (const float*)a.kv_s + b * a.max_entries * int64_t(kD / 64);
+    const uint16_t* raw_seq = (const uint16_t*)a.raw + b * a.n_raw * int64_t(kD);
 
     if (warp >= 4 && warp < kMmaWarp) {
         // ---------------------------------------------------------- producers
@@ -180,9 +183,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) 
         // is unrolled by kLook+1).
         constexpr int kBufs = kLook + 1;
         const int n_steps = 4 * n_tiles;
-        const uint8_t* kv_seq = (const uint8_t*)a.kv + b * a.max_entries * int64_t(kD);
-        const float* kvs_seq = (const float*)a.kv_s + b * a.max_entries * int64_t(kD / 64);
-        const uint16_t* raw_seq = (const uint16_t*)a.raw + b * a.n_raw * int64_t(kD);
         int32_t src[kBufs][kUnits];
         uint4 raw[kBufs][kUnits];
         float sc[kBufs][kUnits];
@@ -335,6 +335,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) 
             vm0 = __ballot_sync(0xffffffffu, s0 < s_hi && (s0 >= n_kv || (j0 >= 0 && j0 < a.max_entries)));
             vm1 = __ballot_sync(0xffffffffu, s1 < s_hi && (s1 >= n_kv || (j1 >= 0 && j1 < a.max_entries)));
         };
+        // Warm L2 with every row this work item reads (pooled FP8 rows with
+        // their scales, bf16 window rows) while the loaders fetch the query:
+        // their gathers then hit L2 instead of waiting on HBM one by one.
+        for (int64_t sl = s_lo + threadIdx.x; sl < s_hi; sl += 128) {
+            const int32_t sr = slot_source(a, row, n_kv, win_lo, p0, sl, s_hi);
+            if (sr < 0) continue;
+            if (sl >= n_kv) {
+                prefetch_l2_bulk(raw_seq + int64_t(sr) * kD, kD * 2);
+            } else {
+                prefetch_l2_bulk(kv_seq + int64_t(sr) * kD, kD);
+                prefetch_l2_bulk(kvs_seq + int64_t(sr) * (kD / 64), (kD / 64) * 4);
+            }
+        }
         int32_t nj0 = 0, nj1 = 0;
         if (n_tiles > 0) load_ids(0, nj0, nj1);
         for (int tile = 0; tile < n_tiles; ++tile) {
@@ -464,6 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) 
             }
         }
     }
+    // the producer and MMA roles run on one lane: reconverge every warp so
+    // that the CTA barrier (an aligned bar.sync) sees whole warps and really
+    // waits for those lanes before TMEM is freed
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == kMmaWarp) tmem_dealloc(tmem, 512);

@@ -335,6 +335,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     }
+    // the producer and MMA roles run on one lane: reconverge every warp so
+    // that the CTA barrier (an aligned bar.sync) sees whole warps and really
+    // waits for those lanes before TMEM is freed
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);

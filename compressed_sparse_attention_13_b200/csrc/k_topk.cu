@@ -8,6 +8,8 @@
 // index order, so ties resolve to the lower index.  -0.0 is folded into +0.0
 // before ranking.  One 1024-thread CTA per query row; rows are read from
 // global memory (an L2-resident score row in the decode path).
+#include <cooperative_groups.h>
+
 #include "kernels.h"
 
 namespace csa {
@@ -19,7 +21,9 @@ __device__ __forceinline__ uint32_t order_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Inclusive block-wide scan of two ints over kTopkThreads threads.
+// Inclusive block-wide scan of two ints over NT threads (a multiple of 32,
+// at most 1024).
+template <int NT = kTopkThreads>
 __device__ __forceinline__ int2 block_scan2(int2 v, int2* warp_tot) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
 #pragma unroll
@@ -31,14 +35,14 @@ __device__ __forceinline__ int2 block_scan2(int2 v, int2* warp_tot) {
     if (lane == 31) warp_tot[wid] = v;
     __syncthreads();
     if (wid == 0) {
-        int2 t = warp_tot[lane];
+        int2 t = lane < NT / 32 ? warp_tot[lane] : make_int2(0, 0);
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int ax = __shfl_up_sync(0xffffffffu, t.x, o);
             const int ay = __shfl_up_sync(0xffffffffu, t.y, o);
             if (lane >= o) { t.x += ax; t.y += ay; }
         }
-        warp_tot[lane] = t;
+        if (lane < NT / 32) warp_tot[lane] = t;
     }
     __syncthreads();
     if (wid > 0) { v.x += warp_tot[wid - 1].x; v.y += warp_tot[wid - 1].y; }
@@ -241,9 +245,148 @@ __global__ void __launch_bounds__(kTopkThreads) topk_smem_kernel(
     write_selection_impl([&](int64_t i) { return keys[i]; }, int64_t(n), prefix, remaining, k, out, warp_tot);
 }
 
+// Few rows (decode): one thread-block cluster of kClu CTAs per row.  CTA r
+// holds keys [r * E * 512, (r + 1) * E * 512) of the row in registers
+// (thread t, slot j: key r * E * 512 + j * 512 + t, so ascending index order
+// is slot-major).  Four 8-bit digit passes as above, except that each CTA
+// counts its own keys and every CTA then sums all kClu histograms through
+// distributed shared memory, so all of them pick the same digit; histograms
+// are double-buffered, so one cluster barrier per pass suffices (a buffer is
+// cleared only after every CTA has passed the barrier that follows its last
+// remote read).  The output offsets of each CTA (keys above T and keys equal
+// to T in lower CTAs) are exchanged the same way.
+namespace cg = cooperative_groups;
+constexpr int kClu = 8;
+constexpr int kCluThreads = 512;
+constexpr int kCluWarps = kCluThreads / 32;
+
+template <int E>
+__global__ void __cluster_dims__(kClu, 1, 1) __launch_bounds__(kCluThreads)
+    topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, int64_t max_blocks,
+                        const int64_t* __restrict__ q_pos, int m, int W, int k,
+                        int32_t* __restrict__ idx) {
+    __shared__ int hist[2][256];
+    __shared__ int2 warp_tot[32];
+    __shared__ int2 cnt[E * kCluWarps];   // per (slot, warp): (keys above T, keys equal to T)
+    __shared__ int2 cta_tot;
+    __shared__ int found_digit, found_above;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int r = int(cluster.block_rank());
+    const int64_t row = blockIdx.x / kClu;
+    const float* s = scores + row * ld;
+    int32_t* out = idx + row * k;
+    const int n = int(min(n_elig(q_pos[row], m, W), max_blocks));
+    const int base = r * E * kCluThreads;
+    if (n <= k) {  // every eligible block is selected (uniform over the cluster)
+        for (int i = base + tid; i < min(k, base + E * kCluThreads); i += kCluThreads)
+            out[i] = i < n ? i : -1;
+        return;
+    }
+    uint32_t key[E];
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+        const int i = base + j * kCluThreads + tid;
+        key[j] = i < n ? order_key(s[i]) : 0u;
+    }
+    if (tid < 256) { hist[0][tid] = 0; hist[1][tid] = 0; }
+    __syncthreads();
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = k;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        int* H = hist[pass & 1];
+        // lanes holding the same digit are merged so that one leader adds
+        // their count (most N(0, s) scores share a few top digits)
+#pragma unroll
+        for (int j = 0; j < E; ++j) {
+            const int i = base + j * kCluThreads + tid;
+            const bool in = i < n && (key[j] & pmask) == prefix;
+            const uint32_t dg = in ? ((key[j] >> shift) & 255u) : 0xFFFFFFFFu;
+            const unsigned same = __match_any_sync(0xffffffffu, dg);
+            if (in && lane == __ffs(same) - 1) atomicAdd(&H[dg], __popc(same));
+        }
+        cluster.sync();
+        // thread t < 256 owns bin 255 - t (bins counted from the top)
+        int c = 0;
+        if (tid < 256) {
+#pragma unroll
+            for (int q = 0; q < kClu; ++q) c += cluster.map_shared_rank(H, q)[255 - tid];
+            hist[(pass + 1) & 1][tid] = 0;  // its last remote reads were before this barrier
+        }
+        const int2 inc = block_scan2<kCluThreads>(make_int2(c, 0), warp_tot);
+        const int above = inc.x - c;
+        if (tid < 256 && above < remaining && remaining <= inc.x) {
+            found_digit = 255 - tid;
+            found_above = above;
+        }
+        __syncthreads();
+        remaining -= found_above;
+        prefix |= uint32_t(found_digit) << shift;
+        pmask |= 0xFFu << shift;
+    }
+    // prefix is the k-th largest key T; the first `remaining` keys equal to T
+    // (in index order) are taken with every key above T.
+    const uint32_t T = prefix;
+    const unsigned lt_mask = (1u << lane) - 1u;
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+        const int i = base + j * kCluThreads + tid;
+        const unsigned gm = __ballot_sync(0xffffffffu, i < n && key[j] > T);
+        const unsigned em = __ballot_sync(0xffffffffu, i < n && key[j] == T);
+        if (lane == 0) cnt[j * kCluWarps + wid] = make_int2(__popc(gm), __popc(em));
+    }
+    __syncthreads();
+    // exclusive offsets of every (slot, warp) in index order, and the CTA total
+    const int2 v = tid < E * kCluWarps ? cnt[tid] : make_int2(0, 0);
+    const int2 vi = block_scan2<kCluThreads>(v, warp_tot);
+    if (tid < E * kCluWarps) cnt[tid] = make_int2(vi.x - v.x, vi.y - v.y);
+    if (tid == E * kCluWarps - 1) cta_tot = vi;
+    cluster.sync();
+    int gt_base = 0, eq_base = 0;
+    for (int q = 0; q < r; ++q) {
+        const int2 t = *cluster.map_shared_rank(&cta_tot, q);
+        gt_base += t.x;
+        eq_base += t.y;
+    }
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+        const int i = base + j * kCluThreads + tid;
+        const bool gt = i < n && key[j] > T, eq = i < n && key[j] == T;
+        const unsigned gm = __ballot_sync(0xffffffffu, gt);
+        const unsigned em = __ballot_sync(0xffffffffu, eq);
+        const int2 off = cnt[j * kCluWarps + wid];
+        const int gt_before = gt_base + off.x + __popc(gm & lt_mask);
+        const int eq_before = eq_base + off.y + __popc(em & lt_mask);
+        if (gt || (eq && eq_before < remaining)) {
+            const int p = gt_before + min(eq_before, remaining);
+            if (p < k) out[p] = int32_t(i);
+        }
+    }
+    cluster.sync();  // keep this CTA's shared memory alive until every remote read is done
+}
+
+template <int E>
+static cudaError_t launch_topk_cluster(const float* scores, int64_t ld, int64_t max_blocks,
+                                       const int64_t* q_pos, int m, int W, int k, int64_t rows,
+                                       int32_t* idx, cudaStream_t s) {
+    topk_cluster_kernel<E><<<unsigned(rows * kClu), kCluThreads, 0, s>>>(scores, ld, max_blocks,
+                                                                        q_pos, m, W, k, idx);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, const int64_t* q_pos,
                         int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
+    // Few rows cannot fill the GPU with one CTA each: give each row a cluster.
+    if (rows <= 2 * kNumSMs / kClu && k <= kClu * kCluThreads && max_blocks <= kClu * kCluThreads * 16) {
+        const int64_t per = ceil_div(max_blocks, kClu * kCluThreads);
+        if (per <= 2) return launch_topk_cluster<2>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
+        if (per <= 4) return launch_topk_cluster<4>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
+        if (per <= 8) return launch_topk_cluster<8>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
+        return launch_topk_cluster<16>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
+    }
     if (max_blocks <= kTopkSmemMax) {
         const size_t sm = size_t(std::max<int64_t>(max_blocks, 1)) * 4;
         cudaError_t e = ensure_smem(topk_smem_kernel, size_t(sm));

@@ -171,9 +171,15 @@ def test_indexer_matches_oracle(idx, HI, dI, n_q, nb, m, W):
 
 
 # --------------------------------------------------------------------- top-k
-@pytest.mark.parametrize("n,k", [(50, 8), (2015, 512), (32736, 512), (5000, 1024), (60000, 1024)])
-def test_topk_matches_oracle_exactly(n, k):
-    rows = 6
+# Few rows take the cluster kernel (one 8-CTA cluster per row, up to 65536
+# scores); many rows take one CTA per row with the row in shared memory (up to
+# 45056 scores) or read from global memory.
+@pytest.mark.parametrize("n,k,rows", [
+    (50, 8, 6), (2015, 512, 6), (32736, 512, 6), (5000, 1024, 6), (60000, 1024, 6),  # cluster
+    (2015, 512, 48), (32736, 512, 48),                                                 # shared memory
+    (60000, 1024, 40), (70000, 1024, 6),                                               # global
+])
+def test_topk_matches_oracle_exactly(n, k, rows):
     s = synth.tensor_np(4, "ts", (rows, n))
     s[1] = np.round(s[1] * 2) / 2          # many exact ties
     s[2, ::3] = 0.0
