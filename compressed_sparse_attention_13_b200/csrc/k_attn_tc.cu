@@ -5,55 +5,70 @@
 // section 架構實現).
 //
 // Shapes: 64 query heads x 512 dims, one KV head; every attended item is its
-// own key and value.  Work item = (query row, split) over a contiguous range
-// of the row's item slots (pooled slots first, then window tokens), taken in
-// tiles of 64 items:
+// own key and value.  A query row's items are cut into 64-item tiles, pooled
+// entries first and then the window tokens, so that no tile mixes the two;
+// work item = (query row, split) over a contiguous range of those tiles:
 //
 //   S[head][item]   = Q[head][:] . K[item][:]           M=64 heads, N=64 items, K=512
 //   P[head][item]   = exp2(S * scale*log2e - m_head)     (one softmax thread per head)
 //   O^T[dim][head] += V^T[dim][item] . P[head][item]^T   4 x (M=128 dims, N=64, K=64)
 //
-// The dequantised tile (E4M3 x fp32 scale -> f16, or the bf16 window -> f16)
-// is stored once as 8 regions of [64 items][64 dims] with 128-byte swizzled
-// rows: the K-major B operand of the first product and the MN-major A operand
-// of the second.  Two tile buffers let the loaders fill tile t+1 while tile t
-// is multiplied.  S (M=64: head h in TMEM lane 32*(h/16) + h%16) is double
-// buffered in TMEM so QK of tile t+1 runs while the softmax works on tile t;
-// O^T takes 4 x 64 columns, one dim per lane.
+// Operands are bf16: the query and the window tokens are used as stored,
+// and each pooled E4M3 x fp32-scale value is rounded once to bf16 (the
+// accumulation is fp32).  A tile is stored once as 8 regions of [64 items]
+// [64 dims] with 128-byte swizzled rows: the K-major B operand of the first
+// product and the MN-major A operand of the second.  Two tile buffers let
+// tile t+1 be fetched and converted while tile t is multiplied.  S (M=64:
+// head h in TMEM lane 32*(h/16) + h%16) is double buffered in TMEM so QK of
+// tile t+1 runs while the softmax works on tile t; O^T takes 4 x 64 columns,
+// one dim per lane.
 //
-// Roles (416 threads): warps 0-3 softmax (lanes 0-15: one head each) and
-// epilogue (all 128 lanes: one dim each per quarter), warps 4-11 load and
-// dequantise with kLook quarter-steps of loads in flight per thread, warp 12
-// issues the MMAs as their inputs become ready: QK of the next tile quarter
-// by quarter, and P.V of the current tile as soon as its P is written, so a
-// slow load of tile t+1 never holds back P.V of tile t.  The running max is kept per head in
-// log2 units and raised only when a tile exceeds it by more than 8, in which
-// case O^T is rescaled in TMEM before the next P.V.  Bounded waits (sm100.cuh).
-#include <type_traits>
+// Data movement: the query (8 tensor copies) and window tiles (8 tensor
+// copies from a [batch][n_raw][512] map; rows past the sequence read as
+// zero) land directly in operand layout.  A pooled tile's FP8 rows land by
+// bulk copy (one per selected row, or one per tile for dense HCA rows) in the
+// upper half of the tile's own buffer and are dequantised in place: dims
+// 0..255 go to the lower half, dims 256..511 are read into registers before
+// any thread overwrites the upper half.
+//
+// Roles (448 threads): warps 0-3 softmax (lanes 0-15: one head each) and
+// epilogue (all 128 lanes: one dim each per quarter), warps 4-11 convert,
+// warp 12 issues the MMAs as their inputs become ready (QK of the next tile,
+// and P.V of the current tile as soon as its P is written), warp 13 resolves
+// the selected ids and issues the copies of each tile as soon as P.V of the
+// tile two back has released its buffer.  The running max is kept per head
+// in log2 units and raised only when a tile exceeds it by more than 8, in
+// which case O^T is rescaled in TMEM before the next P.V.  Bounded waits
+// (sm100.cuh).
+#include <string.h>
 
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tmap.h"
 
 namespace csa {
 
 namespace {
 
 constexpr int kH = 64, kD = 512, kTile = 64;
-constexpr int kProducerWarps = 8;
-constexpr int kProducerThreads = 32 * kProducerWarps;
-constexpr int kMmaWarp = 4 + kProducerWarps;
-constexpr int kThreads = 32 * (kMmaWarp + 1);
-constexpr int kUnits = kTile * 16 / kProducerThreads;  // 8-dim units per thread per quarter (4)
-constexpr int kLook = 2;                               // quarter-steps of loads in flight ahead
+constexpr int kConvWarps = 8;
+constexpr int kConvThreads = 32 * kConvWarps;
+constexpr int kMmaWarp = 4 + kConvWarps;
+constexpr int kIssuerWarp = kMmaWarp + 1;
+constexpr int kThreads = 32 * (kIssuerWarp + 1);
+constexpr int kUnits = kTile * 16 / kConvThreads;  // 8-dim units per thread per quarter (4)
+constexpr int kRawBlk = 4;                         // FP8 rows of a pooled tile: upper half (blocks 4..7)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct SmemAttn {
-    uint8_t kv[2][8][kTile * 128];  // 2 buffers x 8 dim blocks x [64 items][64 f16] (128 KB)
-    uint8_t q[8][kH * 128];         // 8 dim blocks x [64 heads][64 f16] (64 KB)
-    uint8_t p[2][kH * 128];         // 2 buffers x [64 heads][64 items f16] (16 KB)
+    uint8_t kv[2][8][kTile * 128];  // 2 buffers x 8 dim blocks x [64 items][64 bf16] (128 KB)
+    uint8_t q[8][kH * 128];         // 8 dim blocks x [64 heads][64 bf16] (64 KB)
+    uint8_t p[2][kH * 128];         // 2 buffers x [64 heads][64 items bf16] (16 KB)
+    float kvs[2][kTile][kD / 64];   // per buffer: FP8 scales of the tile's items (4 KB)
+    int32_t valid[2][kTile];        // per buffer: item holds data
     float alpha[kH], fin[kH];
-    uint64_t kv_full[2][4], kv_empty[2][4], s_full[2], p_full[2], o_done, q_full;
+    uint64_t raw_full[2], kv_full[2], kv_empty[2], s_full[2], p_full[2], o_done, q_full;
     uint32_t tmem_base;
     int rescale;
 };
@@ -67,18 +82,22 @@ __device__ __forceinline__ void f16x2_of_e4m3x4(uint32_t w, uint32_t& lo, uint32
         : "r"(w));
 }
 
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+// (f16x2 x fp32 scale) -> bf16x2, the product rounded once from fp32
+__device__ __forceinline__ uint32_t bf16x2_scaled(uint32_t h2, float s) {
+    const __half2 h = *reinterpret_cast<const __half2*>(&h2);
+    const float2 f = __half22float2(h);
     uint32_t r;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(f.y * s), "f"(f.x * s));
     return r;
 }
 
-// two bf16 (packed) -> two f16 (packed), rounding to nearest
-__device__ __forceinline__ uint32_t f16x2_of_bf16x2(uint32_t v) {
-    const float lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xFFFF0000u);
-    uint32_t r;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
+// 8 E4M3 values (two words) times their scale -> 8 bf16 (one 16-byte chunk)
+__device__ __forceinline__ uint4 dequant8(uint2 w, float s) {
+    uint32_t f0, f1, f2, f3;
+    f16x2_of_e4m3x4(w.x, f0, f1);
+    f16x2_of_e4m3x4(w.y, f2, f3);
+    return make_uint4(bf16x2_scaled(f0, s), bf16x2_scaled(f1, s), bf16x2_scaled(f2, s),
+                      bf16x2_scaled(f3, s));
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -87,27 +106,22 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// Row of slot `slot` within the sequence's own buffer (pooled entry j, or
-// window row r of the raw buffer), or -1 when the slot is empty or past the
-// range.  Rows fit in 32 bits (checked on the host).
-__device__ __forceinline__ int32_t slot_source(const AttnArgs& a, int64_t row, int64_t n_kv,
-                                               int64_t win_lo, int64_t raw_pos0, int64_t slot,
-                                               int64_t s_hi) {
-    if (slot >= s_hi) return -1;
-    if (slot < n_kv) {
-        const int64_t j = a.idx ? int64_t(a.idx[row * a.k + slot]) : slot;
-        if (j >= a.max_entries) {
-            flag_status(CSA_DEV_BAD_INDEX);
-            return -1;
-        }
-        return j >= 0 ? int32_t(j) : -1;
+// Pooled entry of slot `slot` (< n_kv): its row in the sequence's buffer, or
+// -1 when the slot is empty.  An id past max_entries is flagged and skipped.
+__device__ __forceinline__ int32_t pooled_source(const AttnArgs& a, int64_t row, int64_t slot) {
+    const int64_t j = a.idx ? int64_t(a.idx[row * a.k + slot]) : slot;
+    if (j >= a.max_entries) {
+        flag_status(CSA_DEV_BAD_INDEX);
+        return -1;
     }
-    return int32_t(win_lo + (slot - n_kv) - raw_pos0);
+    return j >= 0 ? int32_t(j) : -1;
 }
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_win,
+                   const AttnArgs a) {
     extern __shared__ uint8_t smem_raw[];
     SmemAttn& S = *reinterpret_cast<SmemAttn*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     using namespace sm100;
@@ -121,19 +135,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) 
     const int64_t p0 = a.raw_pos0[b];
     const int64_t win_lo = max(max(t - a.W + 1, int64_t(0)), p0);
     const int64_t n_win = max(int64_t(0), min(t + 1, p0 + a.n_raw) - win_lo);
-    const int64_t total = n_kv + n_win;
-    const int64_t per = ceil_div(total, a.n_splits);
-    const int64_t s_lo = min(total, split * per), s_hi = min(total, s_lo + per);
-    const int n_tiles = int(ceil_div(s_hi - s_lo, kTile));
+    const int kv_tiles = int(ceil_div(n_kv, kTile)), win_tiles = int(ceil_div(n_win, kTile));
+    const int total_tiles = kv_tiles + win_tiles;
+    const int per = int(ceil_div(total_tiles, a.n_splits));
+    const int tile0 = min(total_tiles, split * per);
+    const int n_tiles = min(total_tiles, tile0 + per) - tile0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            for (int q = 0; q < 4; ++q) { mbar_init(&S.kv_full[i][q], kProducerThreads); mbar_init(&S.kv_empty[i][q], 1); }
+            mbar_init(&S.raw_full[i], 2);  // expect_tx arrival + arrival after the ids / scales
+            mbar_init(&S.kv_full[i], kConvThreads);
+            mbar_init(&S.kv_empty[i], 1);
             mbar_init(&S.s_full[i], 1);
             mbar_init(&S.p_full[i], 128);
         }
         mbar_init(&S.o_done, 1);
-        mbar_init(&S.q_full, kProducerThreads);
+        mbar_init(&S.q_full, 1);
         S.rescale = 0;
         fence_mbar_init();
     }
@@ -143,149 +160,174 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) 
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
     const uint32_t tS = tmem, tO = tmem + 128;  // S[buf]: cols [64 buf, 64 buf + 64); O^T quarter q: [128+64q, 192+64q)
-    const uint8_t* kv_seq = (const uint8_t*)a.kv + b * a.max_entries * int64_t(kD);
-    const float* kvs_seq = (const float*)a.kv_s + b * a.max_entries * int64_t(kD / 64);
-    const uint16_t* raw_seq = (const uint16_t*)a.raw + b * a.n_raw * int64_t(kD);
 
     if (warp >= 4 && warp < kMmaWarp) {
-        // ---------------------------------------------------------- producers
-        const int pt = threadIdx.x - 128;  // 0..kProducerThreads-1
+        // --------------------------------------------------------- converters
+        const int pt = threadIdx.x - 128;  // 0..kConvThreads-1
         const int c = pt & 15;             // 8-dim unit within a 128-dim quarter
         const int e0 = pt >> 4;            // items e0 + 16 u, u < kUnits
-        if (n_tiles > 0) {
-            // query: 64 heads x 512 bf16 -> f16, K-major (A operand): 4096 16-byte
-            // chunks, 8 loads in flight per thread
-            const uint16_t* qg = (const uint16_t*)a.q + row * int64_t(kH) * kD;
-            static_assert((kH * kD / 8) % (8 * kProducerThreads) == 0, "query chunks per batch");
-#pragma unroll 1
-            for (int base = 0; base < kH * kD / 8; base += 8 * kProducerThreads) {
-                uint4 v[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int u = base + pt + kProducerThreads * j;
-                    v[j] = *reinterpret_cast<const uint4*>(qg + (u >> 6) * kD + (u & 63) * 8);
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int u = base + pt + kProducerThreads * j;
-                    const int h = u >> 6, cc = u & 63;
-                    *reinterpret_cast<uint4*>(S.q[cc >> 3] + sw128_offset(h, cc & 7)) =
-                        make_uint4(f16x2_of_bf16x2(v[j].x), f16x2_of_bf16x2(v[j].y),
-                                   f16x2_of_bf16x2(v[j].z), f16x2_of_bf16x2(v[j].w));
-                }
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&S.q_full);
-        }
-        // Software pipeline over (tile, quarter) steps g: the loads of steps
-        // g+1 .. g+kLook are in flight while step g waits for its buffer and is
-        // converted.  Register buffers are compile-time indices (the step loop
-        // is unrolled by kLook+1).
-        constexpr int kBufs = kLook + 1;
-        const int n_steps = 4 * n_tiles;
-        int32_t src[kBufs][kUnits];
-        uint4 raw[kBufs][kUnits];
-        float sc[kBufs][kUnits];
-        auto issue = [&](auto bufc, int g) {
-            constexpr int buf = decltype(bufc)::value;
-            constexpr int prev = (buf + kBufs - 1) % kBufs;
-            const int tile = g >> 2, qt = g & 3;
-            const int64_t slot0 = s_lo + int64_t(tile) * kTile + e0;
-            const int dim0 = 128 * qt + 8 * c;
-#pragma unroll
-            for (int u = 0; u < kUnits; ++u) {
-                // sources are resolved once per tile (quarter 0), then carried
-                const int32_t sr = qt == 0 ? slot_source(a, row, n_kv, win_lo, p0, slot0 + 16 * u, s_hi)
-                                           : src[prev][u];
-                src[buf][u] = sr;
-                raw[buf][u] = make_uint4(0, 0, 0, 0);
-                sc[buf][u] = 0.f;
-                if (sr >= 0) {
-                    if (slot0 + 16 * u >= n_kv) {  // window token (bf16)
-                        raw[buf][u] = *reinterpret_cast<const uint4*>(raw_seq + int64_t(sr) * kD + dim0);
-                    } else {
-                        const uint2 w2 = *reinterpret_cast<const uint2*>(kv_seq + int64_t(sr) * kD + dim0);
-                        raw[buf][u] = make_uint4(w2.x, w2.y, 0, 0);
-                        sc[buf][u] = kvs_seq[int64_t(sr) * (kD / 64) + (dim0 >> 6)];
-                    }
-                }
-            }
-        };
-        auto step = [&](auto bufc, int g) -> bool {
-            constexpr int buf = decltype(bufc)::value;
-            const int tile = g >> 2, qt = g & 3, kb = tile & 1;
-            if (g + kLook < n_steps) issue(std::integral_constant<int, (buf + kLook) % kBufs>{}, g + kLook);
-            if (tile >= 2 && !mbar_wait(&S.kv_empty[kb][qt], uint32_t(((tile >> 1) - 1) & 1))) return false;
-            const int64_t slot0 = s_lo + int64_t(tile) * kTile + e0;
-#pragma unroll
-            for (int u = 0; u < kUnits; ++u) {
-                uint4 o = make_uint4(0, 0, 0, 0);
-                if (src[buf][u] >= 0) {
-                    if (slot0 + 16 * u >= n_kv) {
-                        const uint4 r = raw[buf][u];
-                        o = make_uint4(f16x2_of_bf16x2(r.x), f16x2_of_bf16x2(r.y), f16x2_of_bf16x2(r.z),
-                                       f16x2_of_bf16x2(r.w));
-                    } else {
-                        const float scl = sc[buf][u];
-                        if (scl < 6.103515625e-05f || scl > 146.0f) flag_status(CSA_DEV_RANGE);
-                        const __half2 h2 = __float2half2_rn(scl);
-                        const uint32_t s2 = *reinterpret_cast<const uint32_t*>(&h2);
-                        uint32_t f0, f1, f2, f3;
-                        f16x2_of_e4m3x4(raw[buf][u].x, f0, f1);
-                        f16x2_of_e4m3x4(raw[buf][u].y, f2, f3);
-                        o = make_uint4(hmul2(f0, s2), hmul2(f1, s2), hmul2(f2, s2), hmul2(f3, s2));
-                    }
-                }
-                *reinterpret_cast<uint4*>(S.kv[kb][2 * qt + (c >> 3)] + sw128_offset(e0 + 16 * u, c & 7)) = o;
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&S.kv_full[kb][qt]);
-            return true;
-        };
-        using I0 = std::integral_constant<int, 0>;
-        using I1 = std::integral_constant<int, 1>;
-        using I2 = std::integral_constant<int, 2>;
-        static_assert(kBufs == 3, "the unrolled step loop below assumes three buffers");
-        if (n_steps > 0) issue(I0{}, 0);
-        if (n_steps > 1) issue(I1{}, 1);
         bool ok = true;
-        for (int g = 0; g < n_steps && ok; g += kBufs) {
-            ok = step(I0{}, g);
-            if (ok && g + 1 < n_steps) ok = step(I1{}, g + 1);
-            if (ok && g + 2 < n_steps) ok = step(I2{}, g + 2);
+#pragma unroll 1
+        for (int lt = 0; lt < n_tiles && ok; ++lt) {
+            const int kb = lt & 1;
+            ok = mbar_wait(&S.raw_full[kb], uint32_t((lt >> 1) & 1));
+            if (!ok) break;
+            if (tile0 + lt < kv_tiles) {
+                const uint8_t* raw = S.kv[kb][kRawBlk];  // [64 items][512 E4M3] over blocks 4..7
+                // dims 0..255 -> lower half (the rows sit in the upper half)
+#pragma unroll
+                for (int qt = 0; qt < 2; ++qt)
+#pragma unroll
+                    for (int u = 0; u < kUnits; ++u) {
+                        const int item = e0 + 16 * u;
+                        uint4 o = make_uint4(0, 0, 0, 0);
+                        if (S.valid[kb][item])
+                            o = dequant8(*reinterpret_cast<const uint2*>(raw + kD * item + 128 * qt + 8 * c),
+                                         S.kvs[kb][item][(128 * qt + 8 * c) >> 6]);
+                        *reinterpret_cast<uint4*>(S.kv[kb][2 * qt + (c >> 3)] + sw128_offset(item, c & 7)) = o;
+                    }
+                // dims 256..511: read everything first, then overwrite the upper half
+                uint2 w[2][kUnits];
+                float sc[2][kUnits];
+#pragma unroll
+                for (int qt = 0; qt < 2; ++qt)
+#pragma unroll
+                    for (int u = 0; u < kUnits; ++u) {
+                        const int item = e0 + 16 * u;
+                        const bool v = S.valid[kb][item] != 0;
+                        w[qt][u] = v ? *reinterpret_cast<const uint2*>(raw + kD * item + 128 * (qt + 2) + 8 * c)
+                                     : make_uint2(0, 0);
+                        sc[qt][u] = v ? S.kvs[kb][item][(128 * (qt + 2) + 8 * c) >> 6] : 0.f;
+                    }
+                named_bar(2, kConvThreads);
+#pragma unroll
+                for (int qt = 0; qt < 2; ++qt)
+#pragma unroll
+                    for (int u = 0; u < kUnits; ++u) {
+                        const int item = e0 + 16 * u;
+                        *reinterpret_cast<uint4*>(S.kv[kb][2 * (qt + 2) + (c >> 3)] + sw128_offset(item, c & 7)) =
+                            dequant8(w[qt][u], sc[qt][u]);
+                    }
+            } else {
+                // window tile: already in place; clear rows past the window
+                for (int i = pt; i < kTile * 8 * 8; i += kConvThreads) {
+                    const int item = i >> 6, blk = (i >> 3) & 7, ch = i & 7;
+                    if (!S.valid[kb][item])
+                        *reinterpret_cast<uint4*>(S.kv[kb][blk] + sw128_offset(item, ch)) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&S.kv_full[kb]);
+        }
+    } else if (warp == kIssuerWarp) {
+        // ------------------------------------------------------------- issuer
+        // lane l handles items l and l + 32 of each tile
+        if (n_tiles > 0) {
+            const uint8_t* kv_seq = (const uint8_t*)a.kv + b * a.max_entries * int64_t(kD);
+            const float* kvs_seq = (const float*)a.kv_s + b * a.max_entries * int64_t(kD / 64);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&S.q_full, uint32_t(kH * kD * 2));
+#pragma unroll
+                for (int blk = 0; blk < 8; ++blk)
+                    tma_load_2d(S.q[blk], &map_q, 64 * blk, int32_t(row * kH), &S.q_full);
+            }
+            bool ok = true;
+            int issued = 0;
+#pragma unroll 1
+            for (int lt = 0; lt < n_tiles && ok; ++lt) {
+                const int kb = lt & 1, T = tile0 + lt;
+                if (lt >= 2) ok = mbar_wait(&S.kv_empty[kb], uint32_t(((lt >> 1) - 1) & 1));
+                if (!ok) break;
+                if (T < kv_tiles) {
+                    int32_t sr[2];
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int64_t slot = int64_t(T) * kTile + lane + 32 * h2;
+                        sr[h2] = slot < n_kv ? pooled_source(a, row, slot) : -1;
+                        S.valid[kb][lane + 32 * h2] = sr[h2] >= 0;
+                    }
+                    uint8_t* dst = S.kv[kb][kRawBlk];
+                    if (!a.idx) {
+                        // dense: the tile's rows (and scales) are consecutive
+                        const int64_t j0 = int64_t(T) * kTile;
+                        const uint32_t nv = uint32_t(min(int64_t(kTile), n_kv - j0));
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&S.raw_full[kb], nv * (kD + 32));
+                            bulk_g2s(dst, kv_seq + j0 * kD, nv * kD, &S.raw_full[kb]);
+                            bulk_g2s(&S.kvs[kb][0][0], kvs_seq + j0 * (kD / 64), nv * 32, &S.raw_full[kb]);
+                        }
+                    } else {
+                        uint32_t bytes = (sr[0] >= 0 ? kD : 0) + (sr[1] >= 0 ? kD : 0);
+                        bytes = __reduce_add_sync(0xffffffffu, bytes);
+                        if (lane == 0) mbar_arrive_expect_tx(&S.raw_full[kb], bytes);
+                        __syncwarp();
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2)
+                            if (sr[h2] >= 0)
+                                bulk_g2s(dst + kD * (lane + 32 * h2), kv_seq + int64_t(sr[h2]) * kD, kD,
+                                         &S.raw_full[kb]);
+                        // the scales travel as plain loads while the rows are in flight
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            if (sr[h2] < 0) continue;
+                            const float4* sp = reinterpret_cast<const float4*>(kvs_seq + int64_t(sr[h2]) * (kD / 64));
+                            float4* dp = reinterpret_cast<float4*>(&S.kvs[kb][lane + 32 * h2][0]);
+                            dp[0] = sp[0];
+                            dp[1] = sp[1];
+                        }
+                    }
+                } else {
+                    const int64_t w0 = int64_t(T - kv_tiles) * kTile;
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) S.valid[kb][lane + 32 * h2] = w0 + lane + 32 * h2 < n_win;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&S.raw_full[kb], uint32_t(kTile * kD * 2));
+#pragma unroll
+                        for (int blk = 0; blk < 8; ++blk)
+                            tma_load_3d(S.kv[kb][blk], &map_win, 64 * blk, int32_t(win_lo - p0 + w0),
+                                        int32_t(b), &S.raw_full[kb]);
+                    }
+                }
+                __syncwarp();  // every lane's ids and scales precede lane 0's releasing arrival
+                if (lane == 0) mbar_arrive(&S.raw_full[kb]);
+                ++issued;
+            }
+            // Let every copy still in flight land before the CTA exits (already
+            // the case unless a consumer gave up on a wait).
+            if (lane == 0) {
+                bool drained = mbar_wait(&S.q_full, 0);
+                for (int i = max(0, issued - 2); i < issued && drained; ++i)
+                    drained = mbar_wait(&S.raw_full[i & 1], uint32_t((i >> 1) & 1));
+            }
         }
     } else if (warp == kMmaWarp) {
         // --------------------------------------------------------------- MMA
         if (lane == 0 && n_tiles > 0) {
-            const uint32_t id_qk = instr_desc(0, 0, 0, 0, 64, 64);   // f16: A = Q K-major, B = K K-major
-            const uint32_t id_pv = instr_desc(0, 0, 1, 0, 128, 64);  // f16: A = V^T MN-major, B = P K-major
+            const uint32_t id_qk = instr_desc(1, 1, 0, 0, 64, 64);   // bf16: A = Q K-major, B = K K-major
+            const uint32_t id_pv = instr_desc(1, 1, 1, 0, 128, 64);  // bf16: A = V^T MN-major, B = P K-major
             const uint32_t q0 = smem_u32(S.q[0]);
             bool ok = mbar_wait(&S.q_full, 0);
             // QK(t) may run at most one tile ahead of P.V: it overwrites S[t&1],
             // which the softmax of tile t-2 has finished reading once P.V(t-2)
             // has been issued.  Each wait is a single poll; the loop as a whole
             // is bounded by kWaitNs without progress.
-            int qk_t = 0, qk_q = 0, pv_t = 0;
+            int qk_t = 0, pv_t = 0;
             uint64_t t_last = global_ns();
             while (ok && pv_t < n_tiles) {
                 bool progressed = false;
                 if (qk_t < n_tiles && qk_t <= pv_t + 1) {
                     const int kb = qk_t & 1;
-                    if (mbar_try_wait(&S.kv_full[kb][qk_q], uint32_t((qk_t >> 1) & 1))) {
+                    if (mbar_try_wait(&S.kv_full[kb], uint32_t((qk_t >> 1) & 1))) {
                         tc_fence_after();
                         const uint32_t kv0 = smem_u32(S.kv[kb][0]);
 #pragma unroll
-                        for (int s = 0; s < 8; ++s) {
-                            const int blk = 2 * qk_q + (s >> 2);
+                        for (int s = 0; s < 32; ++s) {
+                            const int blk = s >> 2;
                             mma_f16(tS + 64 * kb, smem_desc(q0 + blk * 8192 + (s & 3) * 32, 16, 1024),
-                                    smem_desc(kv0 + blk * 8192 + (s & 3) * 32, 16, 1024), id_qk,
-                                    (qk_q | s) != 0);
+                                    smem_desc(kv0 + blk * 8192 + (s & 3) * 32, 16, 1024), id_qk, s != 0);
                         }
-                        if (++qk_q == 4) {
-                            mma_commit(&S.s_full[kb]);
-                            qk_q = 0;
-                            ++qk_t;
-                        }
+                        mma_commit(&S.s_full[kb]);
+                        ++qk_t;
                         progressed = true;
                     }
                 }
@@ -294,13 +336,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) 
                     if (mbar_try_wait(&S.p_full[kb], uint32_t((pv_t >> 1) & 1))) {
                         tc_fence_after();
                         const uint32_t kv0 = smem_u32(S.kv[kb][0]), pp = smem_u32(S.p[kb]);
-                        for (int qt = 0; qt < 4; ++qt) {
+#pragma unroll
+                        for (int qt = 0; qt < 4; ++qt)
 #pragma unroll
                             for (int ks = 0; ks < 4; ++ks)
                                 mma_f16(tO + 64 * qt, smem_desc(kv0 + (2 * qt) * 8192 + ks * 2048, 8192, 1024),
                                         smem_desc(pp + ks * 32, 16, 1024), id_pv, (pv_t | ks) != 0);
-                            mma_commit(&S.kv_empty[kb][qt]);
-                        }
+                        mma_commit(&S.kv_empty[kb]);
                         mma_commit(&S.o_done);
                         ++pv_t;
                         progressed = true;
@@ -322,32 +364,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) 
         const float sl2 = a.scale * kLog2e;
         float m_run = -INFINITY, l_run = 0.f;        // per head, log2 units
         bool ok = true;
-        // item validity (slot < s_hi and a pooled id in range, or a window
-        // token) as a 64-bit mask built from two coalesced loads per lane and
-        // ballots; the loads for tile t+1 are issued while tile t is processed
-        auto load_ids = [&](int tt, int32_t& j0, int32_t& j1) {
-            const int64_t s0 = s_lo + int64_t(tt) * kTile + lane, s1 = s0 + 32;
-            j0 = (a.idx && s0 < min(s_hi, n_kv)) ? a.idx[row * a.k + s0] : 0;
-            j1 = (a.idx && s1 < min(s_hi, n_kv)) ? a.idx[row * a.k + s1] : 0;
+        // item validity as a 64-bit mask: pooled slots below n_kv whose id is in
+        // range, or window positions below n_win; the ids of tile t+1 are loaded
+        // while tile t is processed
+        auto load_ids = [&](int lt, int32_t& j0, int32_t& j1) {
+            const int T = tile0 + lt;
+            const int64_t s0 = int64_t(T) * kTile + lane, s1 = s0 + 32;
+            const bool pooled = T < kv_tiles;
+            j0 = (pooled && a.idx && s0 < n_kv) ? a.idx[row * a.k + s0] : 0;
+            j1 = (pooled && a.idx && s1 < n_kv) ? a.idx[row * a.k + s1] : 0;
         };
-        auto mask_of = [&](int tt, int32_t j0, int32_t j1, unsigned& vm0, unsigned& vm1) {
-            const int64_t s0 = s_lo + int64_t(tt) * kTile + lane, s1 = s0 + 32;
-            vm0 = __ballot_sync(0xffffffffu, s0 < s_hi && (s0 >= n_kv || (j0 >= 0 && j0 < a.max_entries)));
-            vm1 = __ballot_sync(0xffffffffu, s1 < s_hi && (s1 >= n_kv || (j1 >= 0 && j1 < a.max_entries)));
-        };
-        // Warm L2 with every row this work item reads (pooled FP8 rows with
-        // their scales, bf16 window rows) while the loaders fetch the query:
-        // their gathers then hit L2 instead of waiting on HBM one by one.
-        for (int64_t sl = s_lo + threadIdx.x; sl < s_hi; sl += 128) {
-            const int32_t sr = slot_source(a, row, n_kv, win_lo, p0, sl, s_hi);
-            if (sr < 0) continue;
-            if (sl >= n_kv) {
-                prefetch_l2_bulk(raw_seq + int64_t(sr) * kD, kD * 2);
+        auto mask_of = [&](int lt, int32_t j0, int32_t j1, unsigned& vm0, unsigned& vm1) {
+            const int T = tile0 + lt;
+            if (T < kv_tiles) {
+                const int64_t s0 = int64_t(T) * kTile + lane, s1 = s0 + 32;
+                vm0 = __ballot_sync(0xffffffffu, s0 < n_kv && j0 >= 0 && j0 < a.max_entries);
+                vm1 = __ballot_sync(0xffffffffu, s1 < n_kv && j1 >= 0 && j1 < a.max_entries);
             } else {
-                prefetch_l2_bulk(kv_seq + int64_t(sr) * kD, kD);
-                prefetch_l2_bulk(kvs_seq + int64_t(sr) * (kD / 64), (kD / 64) * 4);
+                const int64_t w0 = int64_t(T - kv_tiles) * kTile + lane;
+                vm0 = __ballot_sync(0xffffffffu, w0 < n_win);
+                vm1 = __ballot_sync(0xffffffffu, w0 + 32 < n_win);
             }
-        }
+        };
         int32_t nj0 = 0, nj1 = 0;
         if (n_tiles > 0) load_ids(0, nj0, nj1);
         for (int tile = 0; tile < n_tiles; ++tile) {
@@ -377,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) 
             // P.V of the previous tile must be done before P[kb] (read by P.V
             // two tiles back) is rewritten and before O^T is rescaled
             if (ok && tile > 0) ok = mbar_wait(&S.o_done, uint32_t((tile - 1) & 1));
-            // pass 2: P = exp2(x - m) as f16 rows of the K-major B tile, and the sum
+            // pass 2: P = exp2(x - m) as bf16 rows of the K-major B tile, and the sum
             float sum = 0.f;
 #pragma unroll 1
             for (int hf = 0; hf < 2; ++hf) {
@@ -395,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) 
                         uint32_t w4[4];
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            const __half2 hh = __floats2half2_rn(x[8 * ch + 2 * k], x[8 * ch + 2 * k + 1]);
+                            const __nv_bfloat162 hh = __floats2bfloat162_rn(x[8 * ch + 2 * k], x[8 * ch + 2 * k + 1]);
                             w4[k] = *reinterpret_cast<const uint32_t*>(&hh);
                         }
                         *reinterpret_cast<uint4*>(S.p[kb] + sw128_offset(h, 4 * hf + ch)) =
@@ -477,9 +515,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const AttnArgs a) 
             }
         }
     }
-    // the producer and MMA roles run on one lane: reconverge every warp so
-    // that the CTA barrier (an aligned bar.sync) sees whole warps and really
-    // waits for those lanes before TMEM is freed
+    // the issuer and MMA roles run on one lane: reconverge every warp so that
+    // the CTA barrier (an aligned bar.sync) sees whole warps and really waits
+    // for those lanes before TMEM is freed
     __syncwarp();
     tc_fence_before();
     __syncthreads();
@@ -496,10 +534,30 @@ bool attn_tc_rows_fit(int64_t max_entries, int64_t n_raw) {
 
 cudaError_t launch_attn_tc(const AttnArgs& a, int64_t rows, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
+    if (rows * kH >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+    // query [rows * 64][512] bf16 and window tokens [batch][n_raw][512] bf16,
+    // both read as [64 rows][64 dims] boxes with 128-byte swizzle
+    CUtensorMap map_q, map_win;
+    const uint64_t qd[2] = {uint64_t(kD), uint64_t(rows * kH)};
+    const uint64_t qs[1] = {uint64_t(kD) * 2};
+    const uint32_t box2[2] = {64, 64};
+    if (!encode_tile_map(&map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q, qd, qs, box2,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    memset(&map_win, 0, sizeof(map_win));
+    if (a.n_raw > 0) {
+        const int64_t batch = rows / a.n_q;
+        const uint64_t wd[3] = {uint64_t(kD), uint64_t(a.n_raw), uint64_t(batch)};
+        const uint64_t ws[2] = {uint64_t(kD) * 2, uint64_t(a.n_raw) * kD * 2};
+        const uint32_t box3[3] = {64, 64, 1};
+        if (!encode_tile_map(&map_win, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.raw, wd, ws, box3,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
     const size_t sm = sizeof(SmemAttn) + 1024;
     cudaError_t e = ensure_smem(attn_tc_kernel, sm);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<<<dim3(a.n_splits, unsigned(rows)), kThreads, sm, s>>>(a);
+    attn_tc_kernel<<<dim3(a.n_splits, unsigned(rows)), kThreads, sm, s>>>(map_q, map_win, a);
     return cudaGetLastError();
 }
 

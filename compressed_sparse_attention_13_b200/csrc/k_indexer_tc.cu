@@ -39,10 +39,9 @@
 // All waits are bounded (sm100::mbar_wait); after a timed-out wait a role
 // keeps iterating without waiting or touching memory, so every thread still
 // reaches the named and final barriers.
-#include <cuda.h>
-
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tmap.h"
 
 namespace csa {
 
@@ -351,37 +350,13 @@ bool indexer_tc_supported(int fmt, int HI, int dI, int64_t max_blocks, int64_t b
            rows * kHI <= INT32_MAX;
 }
 
-// The driver's tensor-map encoder, looked up through the runtime so that the
-// library does not need libcuda at load time (it loads on hosts without one).
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_tiled_fn() {
-    static EncodeTiledFn fn = []() -> EncodeTiledFn {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
-                                             &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        return reinterpret_cast<EncodeTiledFn>(p);
-    }();
-    return fn;
-}
-
 // 2-D map over [n_rows][64] bytes with 64-byte swizzle and a box of box_rows.
 static bool encode_rows64(CUtensorMap* map, const void* base, int64_t n_rows, int box_rows) {
-    const EncodeTiledFn encode = encode_tiled_fn();
-    if (!encode) return false;
-    const cuuint64_t dims[2] = {cuuint64_t(kKeyBytes), cuuint64_t(n_rows)};
-    const cuuint64_t strides[1] = {cuuint64_t(kKeyBytes)};
-    const cuuint32_t box[2] = {cuuint32_t(kKeyBytes), cuuint32_t(box_rows)};
-    const cuuint32_t elem_strides[2] = {1, 1};
-    return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-                  elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    const uint64_t dims[2] = {uint64_t(kKeyBytes), uint64_t(n_rows)};
+    const uint64_t strides[1] = {uint64_t(kKeyBytes)};
+    const uint32_t box[2] = {uint32_t(kKeyBytes), uint32_t(box_rows)};
+    return encode_tile_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 cudaError_t launch_indexer_tc(const void* qI, const void* qI_s, const float* w, const void* kI,

@@ -108,6 +108,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst_smem, const void* map, int
         : "memory");
 }
 
+// 3-D form of tma_load_2d (coordinates innermost first).
+__device__ __forceinline__ void tma_load_3d(void* dst_smem, const void* map, int32_t x, int32_t y,
+                                            int32_t z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst_smem)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // ------------------------------------------------------------------ TMEM
 // Allocate `ncols` (power of two >= 32) TMEM columns; the base address is
 // written to *dst_smem.  Executed by one full warp.
