@@ -301,7 +301,7 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 1), "unit": "tok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp32 (SIMT) on fp8/mxfp4/bf16 inputs", "data": "synthetic (seeded N(0,1))",
+        "dtype": "mxfp4 indexer + bf16 attention (fp32 accumulate)", "data": "synthetic (seeded N(0,1))",
         "config": {"workload": WORKLOAD, "batch": w.batch, "context": w.n_ctx, "heads": w.H,
                    "head_dim": w.d, "idx_heads": w.HI, "idx_dim": w.dI, "m": w.m, "top_k": w.k,
                    "window": w.W, "kv": "fp8_e4m3_scale64", "indexer": "mxfp4",

@@ -106,17 +106,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// Pooled entry of slot `slot` (< n_kv): its row in the sequence's buffer, or
-// -1 when the slot is empty.  An id past max_entries is flagged and skipped.
-__device__ __forceinline__ int32_t pooled_source(const AttnArgs& a, int64_t row, int64_t slot) {
-    const int64_t j = a.idx ? int64_t(a.idx[row * a.k + slot]) : slot;
-    if (j >= a.max_entries) {
-        flag_status(CSA_DEV_BAD_INDEX);
-        return -1;
-    }
-    return j >= 0 ? int32_t(j) : -1;
-}
-
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -233,19 +222,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             bool ok = true;
             int issued = 0;
+            // software pipeline: the ids of tile lt+1 are loaded during tile lt,
+            // and tile lt's scales are loaded before waiting for its buffer
+            auto load_ids = [&](int lt, int32_t (&j)[2]) {
+                const int T = tile0 + lt;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int64_t slot = int64_t(T) * kTile + lane + 32 * h2;
+                    j[h2] = (T < kv_tiles && a.idx && slot < n_kv) ? a.idx[row * a.k + slot] : -1;
+                }
+            };
+            int32_t jn[2];
+            load_ids(0, jn);
 #pragma unroll 1
             for (int lt = 0; lt < n_tiles && ok; ++lt) {
                 const int kb = lt & 1, T = tile0 + lt;
+                const bool pooled = T < kv_tiles;
+                int32_t sr[2];
+                float4 scl[2][2];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int64_t slot = int64_t(T) * kTile + lane + 32 * h2;
+                    const int64_t j = a.idx ? int64_t(jn[h2]) : slot;
+                    if (pooled && slot < n_kv && j >= a.max_entries) flag_status(CSA_DEV_BAD_INDEX);
+                    sr[h2] = (pooled && slot < n_kv && j >= 0 && j < a.max_entries) ? int32_t(j) : -1;
+                    scl[h2][0] = scl[h2][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (a.idx && sr[h2] >= 0) {
+                        const float4* sp = reinterpret_cast<const float4*>(kvs_seq + int64_t(sr[h2]) * (kD / 64));
+                        scl[h2][0] = sp[0];
+                        scl[h2][1] = sp[1];
+                    }
+                }
+                if (lt + 1 < n_tiles) load_ids(lt + 1, jn);
                 if (lt >= 2) ok = mbar_wait(&S.kv_empty[kb], uint32_t(((lt >> 1) - 1) & 1));
                 if (!ok) break;
-                if (T < kv_tiles) {
-                    int32_t sr[2];
+                if (pooled) {
 #pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        const int64_t slot = int64_t(T) * kTile + lane + 32 * h2;
-                        sr[h2] = slot < n_kv ? pooled_source(a, row, slot) : -1;
-                        S.valid[kb][lane + 32 * h2] = sr[h2] >= 0;
-                    }
+                    for (int h2 = 0; h2 < 2; ++h2) S.valid[kb][lane + 32 * h2] = sr[h2] >= 0;
                     uint8_t* dst = S.kv[kb][kRawBlk];
                     if (!a.idx) {
                         // dense: the tile's rows (and scales) are consecutive
@@ -266,14 +279,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (sr[h2] >= 0)
                                 bulk_g2s(dst + kD * (lane + 32 * h2), kv_seq + int64_t(sr[h2]) * kD, kD,
                                          &S.raw_full[kb]);
-                        // the scales travel as plain loads while the rows are in flight
+                        // the scales were loaded before the wait; store them now
 #pragma unroll
                         for (int h2 = 0; h2 < 2; ++h2) {
-                            if (sr[h2] < 0) continue;
-                            const float4* sp = reinterpret_cast<const float4*>(kvs_seq + int64_t(sr[h2]) * (kD / 64));
                             float4* dp = reinterpret_cast<float4*>(&S.kvs[kb][lane + 32 * h2][0]);
-                            dp[0] = sp[0];
-                            dp[1] = sp[1];
+                            dp[0] = scl[h2][0];
+                            dp[1] = scl[h2][1];
                         }
                     }
                 } else {
@@ -488,7 +499,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_bar(1, 128);
         if (n_tiles > 0 && ok) ok = mbar_wait(&S.o_done, uint32_t((n_tiles - 1) & 1));
         tc_fence_after();
+        // Every P.V has completed, so the two tile buffers (128 KB) are free:
+        // O goes there as [64 heads][512 dims] (fp32 partials, or the final
+        // bf16 output) and leaves in a few bulk stores.
         const int e = sub * 32 + lane;
+        const bool final_out = a.n_splits == 1;
+        float* so32 = reinterpret_cast<float*>(&S.kv[0][0][0]);
+        __nv_bfloat16* so16 = reinterpret_cast<__nv_bfloat16*>(&S.kv[0][0][0]);
         for (int qt = 0; qt < 4; ++qt) {
             const int dim = 128 * qt + e;
 #pragma unroll 1
@@ -500,19 +517,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] = 0.f;
                 }
-                if (a.n_splits == 1) {
-                    __nv_bfloat16* out = (__nv_bfloat16*)a.out + row * int64_t(kH) * kD;
+                if (final_out) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int hh = 32 * hf + i;
-                        out[hh * kD + dim] = __float2bfloat16_rn(o[i] * S.fin[hh]);
+                        so16[hh * kD + dim] = __float2bfloat16_rn(o[i] * S.fin[hh]);
                     }
                 } else {
-                    float* po = a.part_o + (row * a.n_splits + split) * int64_t(kH) * kD;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) po[(32 * hf + i) * kD + dim] = o[i];
+                    for (int i = 0; i < 32; ++i) so32[(32 * hf + i) * kD + dim] = o[i];
                 }
             }
+        }
+        fence_proxy_async_smem();
+        named_bar(1, 128);
+        if (threadIdx.x == 0) {
+            const uint32_t bytes = final_out ? kH * kD * 2 : kH * kD * 4;
+            uint8_t* dst = final_out ? (uint8_t*)a.out + row * int64_t(kH) * kD * 2
+                                     : (uint8_t*)(a.part_o + (row * a.n_splits + split) * int64_t(kH) * kD);
+            const uint8_t* src = &S.kv[0][0][0];
+            for (uint32_t off = 0; off < bytes; off += 16384) bulk_s2g(dst + off, src + off, 16384);
+            bulk_commit_wait_read();
         }
     }
     // the issuer and MMA roles run on one lane: reconverge every warp so that

@@ -84,6 +84,23 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src, uint32
         : "memory");
 }
 
+// 1-D bulk copy shared -> global in the calling thread's bulk group.  Both
+// addresses 16-byte aligned, bytes a multiple of 16; the shared-memory writes
+// it reads must have been made visible to the async proxy first.
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src_smem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(smem_u32(src_smem)), "r"(bytes)
+                 : "memory");
+}
+
+// Close the calling thread's bulk group and wait until every store of it has
+// read its shared-memory source (the writes to global memory complete on their
+// own; they are visible to later kernels).
+__device__ __forceinline__ void bulk_commit_wait_read() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // Ask for `bytes` at src to be brought into L2 (no completion to wait for).
 // src 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {

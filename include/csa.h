@@ -64,7 +64,7 @@ typedef enum csa_status {
 
 /* Bits of the device status word (csa_device_status). */
 #define CSA_DEV_BAD_INDEX 0x1u   /* a selected id >= the entries available; item skipped */
-#define CSA_DEV_RANGE 0x2u       /* a value outside the tensor-core operand range */
+#define CSA_DEV_RANGE 0x2u       /* reserved: no kernel raises it (every stored value is representable) */
 #define CSA_DEV_TIMEOUT 0x4u     /* a kernel's bounded wait gave up; its output is invalid */
 
 /* Per-layer parameters.  Dimensions must be multiples of 64 (head_dim) and
