@@ -322,6 +322,13 @@ def run_ours(args):
         result["hca_decode"] = bench_hca(args, dev, flush, stream, hbm_peak)
         del S
         torch.cuda.empty_cache()
+        for key, leg in (("prefill_8k_bf16", lambda: bench_prefill(dev, flush, stream, bf16_peak)),
+                         ("stack_c4", lambda: bench_stack(dev, flush, stream, hbm_peak))):
+            try:
+                result[key] = leg()
+            except Exception as exc:  # an extra leg must not lose the main line
+                result[key] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+            torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if world > 1:
@@ -370,6 +377,160 @@ def bench_hca(args, dev, flush, stream, hbm_peak):
             "compress": {"workload": "pool 8 x 1M bf16 tokens at m'=128 -> FP8",
                          "ms": round(t_comp, 3), "bytes": comp_bytes,
                          "achieved_gbs": round(comp_bytes / (t_comp / 1e3) / 1e9, 1)}}
+
+
+def _causal_pairs(T, m, W, k, t0=0):
+    """(indexer (query, block) pairs, attended (query, item) pairs) of a chunk
+    of T queries at positions t0 .. t0 + T - 1."""
+    idx = att = 0
+    for t in range(t0, t0 + T):
+        ne = max(0, (t - W) // m)
+        idx += ne
+        att += min(k, ne) + min(W, t + 1)
+    return idx, att
+
+
+def bench_prefill(dev, flush, stream, bf16_peak):
+    """CSA prefill, bf16, T = 8192 (pool the chunk, indexer, top-k, attention)."""
+    import torch
+
+    import compressed_sparse_attention_13_b200 as K
+    from synth.workloads import WORKLOADS, draw_torch
+
+    w = WORKLOADS["csa_prefill_8k_bf16"]
+    B, T, H, d, HI, dI, m, W, k = w.batch, w.n_ctx, w.H, w.d, w.HI, w.dI, w.m, w.W, w.k
+    nb = T // m
+    p = K.params(m, W, k, H, d, HI, dI, w.scale, K.BF16, K.BF16, K.BF16)
+    t_ = {n: draw_torch(w, n, device=dev) for n in ("x", "z", "bias", "q", "qI", "kI", "w", "sinks")}
+    kv = K.empty_stored(K.BF16, B * nb, d, device=dev)
+    qI, kI = K.Stored(K.BF16, t_["qI"]), K.Stored(K.BF16, t_["kI"])
+    out = torch.empty(B, T, H, d, dtype=torch.bfloat16, device=dev)
+    sel = torch.empty(B, T, k, dtype=torch.int32, device=dev)
+    ws = torch.empty(K.csa_workspace_size(p, K.OP_PREFILL, B, T, nb), dtype=torch.uint8, device=dev)
+    fn = lambda: K.csa_prefill(p, B, T, 0, t_["x"], T, 0, t_["z"], t_["bias"], t_["q"], qI, t_["w"], kv,
+                               kI, nb, t_["sinks"], out, sel, ws)
+    times = time_steps(fn, 3, 3, flush, stream)
+    t = statistics.median(times)
+    pi, pa = _causal_pairs(T, m, W, k)
+    flops = B * (pi * 2 * HI * dI + pa * 4 * H * d)
+    tf = flops / (t / 1e3) / 1e12
+    return {"workload": "csa_prefill_8k_bf16", "value": round(B * T / (t / 1e3), 1), "unit": "tok/s",
+            "ms_per_step": round(t, 3), "flop": flops,
+            "roofline": {"kernel": "csa_prefill (CUDA-core bf16 indexer + attention)", "bound": "tensor",
+                         "achieved": round(tf, 2), "peak": bf16_peak, "unit": "TFLOP/s",
+                         "frac": round(tf / bf16_peak, 4)}}
+
+
+def bench_stack(dev, flush, stream, hbm_peak):
+    """Four layers CSA, HCA, CSA, HCA on one sequence at 1M context: a prior
+    cache of 1,044,480 tokens, a 4096-token prefill chunk, then 256 decode steps
+    with incremental pooling (every 4 tokens for CSA, 128 for HCA)."""
+    import math
+
+    import torch
+
+    import compressed_sparse_attention_13_b200 as K
+    from compressed_sparse_attention_13_b200.stack import Layer, LayerSpec
+    from synth import tensor_torch
+
+    PRIOR, CHUNK, STEPS, TOPK, W, H, d, HI, dI = 1_044_480, 4096, 256, 1024, 128, 64, 512, 64, 128
+    scale = 1 / math.sqrt(d)
+    n_new = CHUNK + STEPS
+    g = lambda li, name, shape, std=1.0, dt="f32": tensor_torch(0, f"stack_c4/{li}/{name}", shape, std, dt,
+                                                            device=dev)
+    layers = []
+    for li, kind in enumerate(["csa", "hca", "csa", "hca"]):
+        m = 4 if kind == "csa" else 128
+        p = K.params(m, W, TOPK if kind == "csa" else 1, H, d, HI, dI, scale, K.BF16, K.FP8_S64, K.MXFP4)
+        L = Layer(LayerSpec(kind, p, PRIOR, n_new), dev)
+        K.csa_quantize(g(li, "prior_kv", (PRIOR // m, d)), K.Stored(K.FP8_S64, L.kv.data[:PRIOR // m],
+                                                                    L.kv.scales[:PRIOR // m]))
+        L.set_prior_window(g(li, "x_prior", (W - 1, d), dt="bf16"))
+        inp = dict(kind=kind, L=L, x=g(li, "x", (n_new, d), dt="bf16"), z=g(li, "z", (n_new, d), dt="bf16"),
+                   bias=g(li, "bias", (m, d), 0.1), q=g(li, "q", (n_new, H, d), dt="bf16"),
+                   sinks=g(li, "sinks", (H,)), out=torch.empty(n_new, H, d, dtype=torch.bfloat16, device=dev),
+                   sel=torch.empty(n_new, TOPK, dtype=torch.int32, device=dev))
+        if kind == "csa":
+            K.csa_quantize(g(li, "prior_kI", (PRIOR // m, dI)),
+                           K.Stored(K.MXFP4, L.kI.data[:PRIOR // m], L.kI.scales[:PRIOR // m]))
+            qI = K.empty_stored(K.MXFP4, n_new * HI, dI, device=dev)
+            K.csa_quantize(g(li, "qI", (n_new * HI, dI)), qI)
+            inp.update(xI=g(li, "xI", (n_new, dI), dt="bf16"), zI=g(li, "zI", (n_new, dI), dt="bf16"),
+                       biasI=g(li, "biasI", (m, dI), 0.1), qI=qI, w=g(li, "w", (n_new, HI), 0.1))
+        layers.append(inp)
+    torch.cuda.synchronize()
+
+    def rows(st, a, b):
+        return K.Stored(st.fmt, st.data[a:b], st.scales[a:b])
+
+    # prefill chunk (all four layers)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush.zero_()
+    e0.record(stream)
+    for ly in layers:
+        L, csa = ly["L"], ly["kind"] == "csa"
+        L.append(ly["x"][:CHUNK], ly["z"][:CHUNK], ly["xI"][:CHUNK] if csa else None,
+                 ly["zI"][:CHUNK] if csa else None)
+        L.prefill(CHUNK, ly["q"][:CHUNK], rows(ly["qI"], 0, CHUNK * HI) if csa else None,
+                  ly["w"][:CHUNK] if csa else None, ly["sinks"], ly["out"][:CHUNK],
+                  ly["sel"][:CHUNK] if csa else None, ly["bias"], ly.get("biasI"))
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_prefill = e0.elapsed_time(e1)
+    assert K.csa_device_status(reset=True) == 0
+    # decode steps: one eager pass (loads every kernel), then the same steps
+    # captured once in a graph and replayed (appends and pooling rewrite the
+    # same rows, so a replay recomputes the same outputs)
+    qpos = torch.arange(PRIOR + CHUNK, PRIOR + n_new, dtype=torch.int64, device=dev)
+    start = [ly["L"].state() for ly in layers]
+
+    def steps():
+        for s in range(STEPS):
+            i = CHUNK + s
+            for ly in layers:
+                L, csa = ly["L"], ly["kind"] == "csa"
+                L.append(ly["x"][i:i + 1], ly["z"][i:i + 1], ly["xI"][i:i + 1] if csa else None,
+                         ly["zI"][i:i + 1] if csa else None)
+                L.decode(ly["q"][i], rows(ly["qI"], i * HI, (i + 1) * HI) if csa else None,
+                         ly["w"][i] if csa else None, ly["sinks"], ly["out"][i], ly["sel"][i] if csa else None,
+                         ly["bias"], ly.get("biasI"), q_pos=qpos[s:s + 1])
+
+    steps()
+    torch.cuda.synchronize()
+    assert K.csa_device_status(reset=True) == 0
+    for ly, st in zip(layers, start):
+        ly["L"].restore(st)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        steps()
+    dec = []
+    for _ in range(3):
+        flush.zero_()
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dec.append(e0.elapsed_time(e1))
+    assert K.csa_device_status(reset=True) == 0
+    del graph
+    t_dec = statistics.median(dec) / STEPS
+    # algorithmic bytes of one decode step (four layers)
+    by = 0
+    for ly in layers:
+        t = PRIOR + CHUNK + STEPS // 2
+        if ly["kind"] == "csa":
+            ne = (t - W) // 4
+            by += ne * (64 + 4) + 2 * ne * 4 + TOPK * (d + 32) + W * d * 2 + 2 * H * d * 2
+        else:
+            ne = (t - W) // 128
+            by += ne * (d + 32) + W * d * 2 + 2 * H * d * 2
+    gbs = by / (t_dec / 1e3) / 1e9
+    return {"workload": "csa_hca_stack_1m_4layers", "prior_tokens": PRIOR, "chunk": CHUNK, "decode_steps": STEPS,
+            "prefill_ms": round(t_prefill, 3), "prefill_tok_s": round(CHUNK / (t_prefill / 1e3), 1),
+            "decode_us_per_step": round(t_dec * 1e3, 2), "decode_tok_s": round(1 / (t_dec / 1e3), 1),
+            "decode_step_bytes": by,
+            "roofline": {"kernel": "decode step (4 layers)", "bound": "hbm", "achieved": round(gbs, 1),
+                         "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4)}}
 
 
 # ------------------------------------------------------------- CPU oracle

@@ -115,9 +115,12 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
     a.part_ml = (float2*)((char*)ws + plan.part_o_bytes);
     const bool tc = attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim) &&
                     attn_tc_rows_fit(max_entries, n_raw);
-    int st = cuda_status(tc ? launch_attn_tc(a, rows, s) : launch_attn_simt(p->act_fmt, p->kv_fmt, a, rows, s));
+    a.fused_combine = 0;
+    bool combined = false;
+    int st = cuda_status(tc ? launch_attn_tc(a, rows, s, &combined)
+                            : launch_attn_simt(p->act_fmt, p->kv_fmt, a, rows, s));
     if (st) return st;
-    if (plan.n_splits > 1)
+    if (plan.n_splits > 1 && !combined)
         st = cuda_status(launch_combine(p->act_fmt, p->n_heads, p->head_dim, plan.n_splits, rows,
                                         a.part_o, a.part_ml, sinks, out, s));
     return st;
@@ -164,7 +167,10 @@ int csa_compress(const csa_params* p, int32_t d, const void* x, const void* z, c
     if (n_tokens == 0) return CSA_OK;
     if (!x || !z || !bias || !out) return CSA_ERR_ARG;
     if ((out_fmt == CSA_FP8_S64 || out_fmt == CSA_MXFP4) && !out_scales) return CSA_ERR_ARG;
-    if (!aligned16(x) || !aligned16(z) || !aligned16(bias) || !aligned16(out) || !aligned16(out_scales))
+    // scales are stored one by one (fp32 for FP8_S64, one byte for MXFP4), so
+    // a single pooled row can be appended at any index
+    const bool scales_ok = out_fmt != CSA_FP8_S64 || (reinterpret_cast<uintptr_t>(out_scales) & 3) == 0;
+    if (!aligned16(x) || !aligned16(z) || !aligned16(bias) || !aligned16(out) || !scales_ok)
         return CSA_ERR_ALIGN;
     return cuda_status(launch_compress(p->act_fmt, out_fmt, x, z, bias, n_tokens, p->m, d, out,
                                        out_scales, (cudaStream_t)stream));

@@ -42,6 +42,9 @@
 // (sm100.cuh).
 #include <string.h>
 
+#include <cooperative_groups.h>
+#include <mutex>
+
 #include "kernels.h"
 #include "sm100.cuh"
 #include "tmap.h"
@@ -68,6 +71,8 @@ struct SmemAttn {
     float kvs[2][kTile][kD / 64];   // per buffer: FP8 scales of the tile's items (4 KB)
     int32_t valid[2][kTile];        // per buffer: item holds data
     float alpha[kH], fin[kH];
+    float2 ml[kH];                  // cluster combine: this split's (max in log2 units, sum) per head
+    float cw[8][kH], cinv[kH];      // cluster combine: weight of each split, 1 / denominator
     uint64_t raw_full[2], kv_full[2], kv_empty[2], s_full[2], p_full[2], o_done, q_full;
     uint32_t tmem_base;
     int rescale;
@@ -490,6 +495,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     den = l_run * f + ex2(sg - M);
                 }
                 S.fin[h] = den > 0.f ? f / den : 0.f;
+            } else if (a.fused_combine) {
+                S.ml[h] = make_float2(m_run, l_run);
+                S.fin[h] = 1.f;
             } else {
                 const int64_t item = row * a.n_splits + split;
                 a.part_ml[item * kH + h] = make_float2(m_run == -INFINITY ? -INFINITY : m_run / kLog2e, l_run);
@@ -531,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         named_bar(1, 128);
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == 0 && !a.fused_combine) {
             const uint32_t bytes = final_out ? kH * kD * 2 : kH * kD * 4;
             uint8_t* dst = final_out ? (uint8_t*)a.out + row * int64_t(kH) * kD * 2
                                      : (uint8_t*)(a.part_o + (row * a.n_splits + split) * int64_t(kH) * kD);
@@ -547,6 +555,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+    if (a.fused_combine) {
+        // The splits of this row form the cluster; each has staged its fp32 O
+        // ([64 heads][512 dims] in its tile buffers) and (m, l) per head.  CTA
+        // r combines an r-th of the output, reading every split's partial
+        // through distributed shared memory, and writes the final bf16.
+        namespace cg = cooperative_groups;
+        cg::cluster_group cl = cg::this_cluster();
+        const int ns = a.n_splits, r = int(cl.block_rank());
+        cl.sync();
+        if (threadIdx.x < kH) {
+            const int hh = threadIdx.x;
+            float m[8], l[8];
+            float M = a.sinks ? a.sinks[hh] * kLog2e : -INFINITY;
+            for (int q = 0; q < ns; ++q) {
+                const float2 v = cl.map_shared_rank(&S.ml[0], q)[hh];
+                m[q] = v.x;
+                l[q] = v.y;
+                M = fmaxf(M, v.x);
+            }
+            float den = 0.f;
+            for (int q = 0; q < ns; ++q) {
+                const float wq = m[q] == -INFINITY ? 0.f : ex2(m[q] - M);
+                S.cw[q][hh] = wq;
+                den += wq * l[q];
+            }
+            if (a.sinks) den += ex2(a.sinks[hh] * kLog2e - M);
+            S.cinv[hh] = den > 0.f ? 1.f / den : 0.f;
+        }
+        __syncthreads();
+        constexpr int n4 = kH * kD / 4;
+        const int lo = r * n4 / ns, hi = (r + 1) * n4 / ns;
+        const float4* part = reinterpret_cast<const float4*>(&S.kv[0][0][0]);
+        __nv_bfloat16* out = (__nv_bfloat16*)a.out + row * int64_t(kH) * kD;
+        for (int i = lo + threadIdx.x; i < hi; i += kThreads) {
+            const int hh = (4 * i) / kD;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int q = 0; q < ns; ++q) {
+                const float4 v = cl.map_shared_rank(part, q)[i];
+                const float wq = S.cw[q][hh];
+                acc.x += wq * v.x; acc.y += wq * v.y; acc.z += wq * v.z; acc.w += wq * v.w;
+            }
+            const float inv = S.cinv[hh];
+            const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+            const __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+            uint2 pk;
+            pk.x = *reinterpret_cast<const uint32_t*>(&lo2);
+            pk.y = *reinterpret_cast<const uint32_t*>(&hi2);
+            *reinterpret_cast<uint2*>(out + 4 * int64_t(i)) = pk;
+        }
+        cl.sync();  // keep this CTA's shared memory alive until every remote read is done
+    }
 }
 
 bool attn_tc_supported(int act, int kvf, int H, int D) {
@@ -557,8 +616,29 @@ bool attn_tc_rows_fit(int64_t max_entries, int64_t n_raw) {
     return max_entries < (int64_t(1) << 31) && n_raw < (int64_t(1) << 31);
 }
 
-cudaError_t launch_attn_tc(const AttnArgs& a, int64_t rows, cudaStream_t s) {
+// Whether clusters of cfg's size can be scheduled for this kernel on the
+// current device (queried once per device and size).
+static bool cluster_fits(const cudaLaunchConfig_t& cfg) {
+    static std::mutex mu;
+    static int known[64][9];  // 0 unknown, 1 yes, 2 no
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    const int n = int(cfg.gridDim.x);
+    std::lock_guard<std::mutex> lock(mu);
+    if (known[dev][n] == 0) {
+        int n_clusters = 0;
+        const bool ok = cudaOccupancyMaxActiveClusters(&n_clusters, attn_tc_kernel, &cfg) == cudaSuccess &&
+                        n_clusters > 0;
+        if (!ok) (void)cudaGetLastError();
+        known[dev][n] = ok ? 1 : 2;
+    }
+    return known[dev][n] == 1;
+}
+
+cudaError_t launch_attn_tc(const AttnArgs& a_in, int64_t rows, cudaStream_t s, bool* combined) {
+    *combined = false;
     if (rows == 0) return cudaSuccess;
+    AttnArgs a = a_in;
     if (rows * kH >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
     // query [rows * 64][512] bf16 and window tokens [batch][n_raw][512] bf16,
     // both read as [64 rows][64 dims] boxes with 128-byte swizzle
@@ -582,8 +662,32 @@ cudaError_t launch_attn_tc(const AttnArgs& a, int64_t rows, cudaStream_t s) {
     const size_t sm = sizeof(SmemAttn) + 1024;
     cudaError_t e = ensure_smem(attn_tc_kernel, sm);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<<<dim3(a.n_splits, unsigned(rows)), kThreads, sm, s>>>(map_q, map_win, a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.n_splits, unsigned(rows));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = sm;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(a.n_splits);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    // The splits of a row combine inside the kernel when they fit one portable
+    // cluster and such clusters can be scheduled; otherwise launch_combine runs.
+    if (a.n_splits >= 2 && a.n_splits <= 8) {
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cluster_fits(cfg)) {
+            a.fused_combine = 1;
+            e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, map_q, map_win, a);
+            if (e == cudaSuccess) *combined = true;
+            return e;
+        }
+        cfg.attrs = nullptr;
+        cfg.numAttrs = 0;
+    }
+    a.fused_combine = 0;
+    return cudaLaunchKernelEx(&cfg, attn_tc_kernel, map_q, map_win, a);
 }
 
 }  // namespace csa

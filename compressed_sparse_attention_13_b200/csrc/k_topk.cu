@@ -245,8 +245,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_smem_kernel(
     write_selection_impl([&](int64_t i) { return keys[i]; }, int64_t(n), prefix, remaining, k, out, warp_tot);
 }
 
-// Few rows (decode): one thread-block cluster of kClu CTAs per row.  CTA r
-// holds keys [r * E * 512, (r + 1) * E * 512) of the row in registers
+// Few rows (decode): one thread-block cluster of kClu CTAs per row (rows of
+// up to 8 x 512 x 72 = 294,912 scores).  CTA r holds keys
+// [r * E * 512, (r + 1) * E * 512) of the row in registers
 // (thread t, slot j: key r * E * 512 + j * 512 + t, so ascending index order
 // is slot-major).  Four 8-bit digit passes as above, except that each CTA
 // counts its own keys and every CTA then sums all kClu histograms through
@@ -338,11 +339,27 @@ __global__ void __cluster_dims__(kClu, 1, 1) __launch_bounds__(kCluThreads)
         if (lane == 0) cnt[j * kCluWarps + wid] = make_int2(__popc(gm), __popc(em));
     }
     __syncthreads();
-    // exclusive offsets of every (slot, warp) in index order, and the CTA total
-    const int2 v = tid < E * kCluWarps ? cnt[tid] : make_int2(0, 0);
-    const int2 vi = block_scan2<kCluThreads>(v, warp_tot);
-    if (tid < E * kCluWarps) cnt[tid] = make_int2(vi.x - v.x, vi.y - v.y);
-    if (tid == E * kCluWarps - 1) cta_tot = vi;
+    // exclusive offsets of every (slot, warp) in index order, and the CTA
+    // total; thread t scans the R consecutive entries [t R, t R + R)
+    constexpr int kEntries = E * kCluWarps, R = (kEntries + kCluThreads - 1) / kCluThreads;
+    int2 mine[R], sum = make_int2(0, 0);
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        const int e = tid * R + i;
+        mine[i] = e < kEntries ? cnt[e] : make_int2(0, 0);
+        sum.x += mine[i].x;
+        sum.y += mine[i].y;
+    }
+    const int2 vi = block_scan2<kCluThreads>(sum, warp_tot);
+    int2 run = make_int2(vi.x - sum.x, vi.y - sum.y);
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        const int e = tid * R + i;
+        if (e < kEntries) cnt[e] = run;
+        run.x += mine[i].x;
+        run.y += mine[i].y;
+    }
+    if (tid == kCluThreads - 1) cta_tot = vi;
     cluster.sync();
     int gt_base = 0, eq_base = 0;
     for (int q = 0; q < r; ++q) {
@@ -380,12 +397,14 @@ cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, con
                         int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
     // Few rows cannot fill the GPU with one CTA each: give each row a cluster.
-    if (rows <= 2 * kNumSMs / kClu && k <= kClu * kCluThreads && max_blocks <= kClu * kCluThreads * 16) {
+    if (rows <= 2 * kNumSMs / kClu && k <= kClu * kCluThreads && max_blocks <= kClu * kCluThreads * 72) {
         const int64_t per = ceil_div(max_blocks, kClu * kCluThreads);
         if (per <= 2) return launch_topk_cluster<2>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
         if (per <= 4) return launch_topk_cluster<4>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
         if (per <= 8) return launch_topk_cluster<8>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
-        return launch_topk_cluster<16>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
+        if (per <= 16) return launch_topk_cluster<16>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
+        if (per <= 32) return launch_topk_cluster<32>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
+        return launch_topk_cluster<72>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
     }
     if (max_blocks <= kTopkSmemMax) {
         const size_t sm = size_t(std::max<int64_t>(max_blocks, 1)) * 4;

@@ -23,6 +23,8 @@ struct AttnArgs {
     void* out;                // final output when n_splits == 1
     float* part_o;            // [rows][n_splits][H][D]
     float2* part_ml;          // [rows][n_splits][H] (running max, running sum)
+    int fused_combine;        // tensor-core kernel: the splits of a row form a cluster and
+                              // combine through distributed shared memory (set by the launcher)
 };
 
 cudaError_t launch_compress(int in_fmt, int out_fmt, const void* x, const void* z,
@@ -44,7 +46,9 @@ cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, con
                         int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s);
 bool attn_tc_supported(int act, int kvf, int H, int D);
 bool attn_tc_rows_fit(int64_t max_entries, int64_t n_raw);
-cudaError_t launch_attn_tc(const AttnArgs& a, int64_t rows, cudaStream_t s);
+// Sets *combined when the splits were combined inside the kernel (no
+// launch_combine needed).
+cudaError_t launch_attn_tc(const AttnArgs& a, int64_t rows, cudaStream_t s, bool* combined);
 cudaError_t launch_attn_simt(int act, int kvf, const AttnArgs& a, int64_t rows, cudaStream_t s);
 bool attn_simt_supported(int act, int kvf, int H, int D);
 cudaError_t launch_combine(int act, int H, int D, int n_splits, int64_t rows, const float* part_o,

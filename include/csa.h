@@ -96,7 +96,9 @@ typedef struct csa_params {
  *   x, z:      [n_tokens][d] in p->act_fmt; n_tokens a multiple of p->m
  *   bias:      float [p->m][d]
  *   out:       [n_tokens/m][d] in out_fmt; out_scales as the format needs
- *              (NULL for F32 / BF16)
+ *              (NULL for F32 / BF16).  out_scales needs only 4-byte alignment
+ *              (FP8_S64) or none (MXFP4), so that one pooled row can be
+ *              written at any row index of a cache
  *   d:         channels (a multiple of 64); p->head_dim is not used, so the
  *              same call pools indexer keys (d = idx_dim)
  * ------------------------------------------------------------------------ */

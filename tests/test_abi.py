@@ -72,6 +72,8 @@ def test_host_side_argument_errors_need_no_gpu():
     assert lib.csa_compress(P, 64, fake, fake, fake, 8, K.FP8_S64, fake, None, None) == -1
     # misaligned input
     assert lib.csa_compress(P, 64, odd, fake, fake, 8, K.F32, fake, None, None) == -2
+    # FP8 scales must be 4-byte aligned (MXFP4 scales are single bytes: any address)
+    assert lib.csa_compress(P, 64, fake, fake, fake, 8, K.FP8_S64, fake, C.c_void_p(0x1002), None) == -2
     # unknown quantisation format
     assert lib.csa_quantize(7, fake, 4, 64, fake, fake, None) == -1
     # ld_scores smaller than max_blocks

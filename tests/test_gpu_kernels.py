@@ -171,13 +171,14 @@ def test_indexer_matches_oracle(idx, HI, dI, n_q, nb, m, W):
 
 
 # --------------------------------------------------------------------- top-k
-# Few rows take the cluster kernel (one 8-CTA cluster per row, up to 65536
-# scores); many rows take one CTA per row with the row in shared memory (up to
-# 45056 scores) or read from global memory.
+# Few rows take the cluster kernel (one 8-CTA cluster per row, up to 294,912
+# scores); many rows, or longer rows, take one CTA per row with the row in
+# shared memory (up to 45056 scores) or read from global memory.
 @pytest.mark.parametrize("n,k,rows", [
     (50, 8, 6), (2015, 512, 6), (32736, 512, 6), (5000, 1024, 6), (60000, 1024, 6),  # cluster
     (2015, 512, 48), (32736, 512, 48),                                                 # shared memory
-    (60000, 1024, 40), (70000, 1024, 6),                                               # global
+    (70000, 1024, 6), (250000, 1024, 6),                                              # cluster, large
+    (60000, 1024, 40), (300000, 512, 6),                                               # global
 ])
 def test_topk_matches_oracle_exactly(n, k, rows):
     s = synth.tensor_np(4, "ts", (rows, n))
@@ -212,9 +213,14 @@ def _attn_case(act, kvf, H, d, batch, n_q, n_ent, W, k, m, seed, scale):
     return qv, ent, raw, n_raw, sinks, q_pos, raw_pos0
 
 
+# 2 x 12 and 2 x 20 query rows split each row 6 and 3 ways on the tensor-core
+# path, where the splits of a row form a cluster and combine in the kernel;
+# 6 rows split 10 ways and use the separate combine kernel.
 @pytest.mark.parametrize("act,kvf,H,d,n_q,n_ent,W,k,m", [
     ("f32", "f32", 8, 64, 20, 256, 64, 16, 4),
     ("bf16", "fp8", 64, 512, 3, 700, 128, 512, 4),
+    ("bf16", "fp8", 64, 512, 12, 700, 128, 512, 4),
+    ("bf16", "fp8", 64, 512, 20, 400, 128, 256, 4),
     ("bf16", "bf16", 64, 512, 4, 300, 128, 64, 4),
 ])
 def test_sparse_attention_matches_oracle(act, kvf, H, d, n_q, n_ent, W, k, m):
