@@ -97,7 +97,7 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
                     const void* kv_s, int64_t max_entries, const int32_t* idx, const void* raw,
                     int64_t n_raw, const int64_t* raw_pos0, const int64_t* q_pos,
                     const float* sinks, void* out, void* ws, size_t ws_bytes, int64_t items_per_row,
-                    cudaStream_t s) {
+                    cudaStream_t s, bool pdl = false) {
     const int64_t rows = int64_t(batch) * n_q;
     if (!attn_simt_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim) &&
         !attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim))
@@ -117,12 +117,13 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
                     attn_tc_rows_fit(max_entries, n_raw);
     a.fused_combine = 0;
     bool combined = false;
-    int st = cuda_status(tc ? launch_attn_tc(a, rows, s, &combined)
+    int st = cuda_status(tc ? launch_attn_tc(a, rows, s, &combined, pdl)
                             : launch_attn_simt(p->act_fmt, p->kv_fmt, a, rows, s));
     if (st) return st;
+    // the combine always follows this function's own attention launch
     if (plan.n_splits > 1 && !combined)
         st = cuda_status(launch_combine(p->act_fmt, p->n_heads, p->head_dim, plan.n_splits, rows,
-                                        a.part_o, a.part_ml, sinks, out, s));
+                                        a.part_o, a.part_ml, sinks, out, s, /*pdl=*/true));
     return st;
 }
 
@@ -210,23 +211,46 @@ int indexer_score(const csa_params* p, int32_t batch, int32_t n_q, const void* q
                                            (cudaStream_t)stream));
 }
 
-int topk_select(const csa_params* p, int32_t batch, int32_t n_q, const float* scores,
-                int64_t ld_scores, int64_t max_blocks, const int64_t* q_pos, int32_t* idx,
-                csa_stream_t stream) {
+static int topk_impl(const csa_params* p, int32_t batch, int32_t n_q, const float* scores,
+                     int64_t ld_scores, int64_t max_blocks, const int64_t* q_pos, int32_t* idx,
+                     csa_stream_t stream, bool pdl) {
     if (!p || p->m <= 0 || p->window < 0 || p->top_k <= 0) return CSA_ERR_ARG;
     if (batch < 0 || n_q < 0 || max_blocks < 0 || ld_scores < max_blocks) return CSA_ERR_ARG;
     if (max_blocks > INT32_MAX) return CSA_ERR_UNSUPPORTED;
     if (batch == 0 || n_q == 0) return CSA_OK;
     if (!q_pos || !idx || (max_blocks > 0 && !scores)) return CSA_ERR_ARG;
     return cuda_status(launch_topk(scores, ld_scores, max_blocks, q_pos, p->m, p->window, p->top_k,
-                                   int64_t(batch) * n_q, idx, (cudaStream_t)stream));
+                                   int64_t(batch) * n_q, idx, (cudaStream_t)stream, pdl));
 }
+
+int topk_select(const csa_params* p, int32_t batch, int32_t n_q, const float* scores,
+                int64_t ld_scores, int64_t max_blocks, const int64_t* q_pos, int32_t* idx,
+                csa_stream_t stream) {
+    return topk_impl(p, batch, n_q, scores, ld_scores, max_blocks, q_pos, idx, stream, false);
+}
+
+static int sparse_attn_impl(const csa_params* p, int32_t batch, int32_t n_q, const void* q,
+                            const void* kv, const void* kv_scales, int64_t max_entries,
+                            const int32_t* idx, const void* raw, int64_t n_raw,
+                            const int64_t* raw_pos0, const int64_t* q_pos, const float* sinks,
+                            void* out, void* workspace, size_t ws_bytes, csa_stream_t stream,
+                            bool pdl);
 
 int sparse_mqa_attn(const csa_params* p, int32_t batch, int32_t n_q, const void* q, const void* kv,
                     const void* kv_scales, int64_t max_entries, const int32_t* idx,
                     const void* raw, int64_t n_raw, const int64_t* raw_pos0,
                     const int64_t* q_pos, const float* sinks, void* out, void* workspace,
                     size_t ws_bytes, csa_stream_t stream) {
+    return sparse_attn_impl(p, batch, n_q, q, kv, kv_scales, max_entries, idx, raw, n_raw, raw_pos0,
+                            q_pos, sinks, out, workspace, ws_bytes, stream, false);
+}
+
+static int sparse_attn_impl(const csa_params* p, int32_t batch, int32_t n_q, const void* q,
+                            const void* kv, const void* kv_scales, int64_t max_entries,
+                            const int32_t* idx, const void* raw, int64_t n_raw,
+                            const int64_t* raw_pos0, const int64_t* q_pos, const float* sinks,
+                            void* out, void* workspace, size_t ws_bytes, csa_stream_t stream,
+                            bool pdl) {
     int st = check_params(p, false, true);
     if (st) return st;
     if (p->top_k <= 0 || batch < 0 || n_q < 0 || max_entries < 0) return CSA_ERR_ARG;
@@ -236,7 +260,7 @@ int sparse_mqa_attn(const csa_params* p, int32_t batch, int32_t n_q, const void*
     if (st) return st;
     return run_attn(p, batch, n_q, q, kv, kv_scales, max_entries, idx, raw, n_raw, raw_pos0, q_pos,
                     sinks, out, workspace, ws_bytes, int64_t(p->top_k) + p->window,
-                    (cudaStream_t)stream);
+                    (cudaStream_t)stream, pdl);
 }
 
 int hca_attn(const csa_params* p, int32_t batch, int32_t n_q, const void* q, const void* kv,
@@ -299,10 +323,13 @@ int csa_decode(const csa_params* p, int32_t batch, const void* q, const void* qI
     st = indexer_score(p, batch, 1, qI, qI_scales, w, kI, kI_scales, max_blocks, q_pos, scores, ld,
                        stream);
     if (st) return st;
-    st = topk_select(p, batch, 1, scores, ld, max_blocks, q_pos, sel, stream);
+    // (Launching top-k and attention as programmatic dependents of the kernel
+    // before them measured slower on this step: their early CTAs take SM
+    // slots from the running kernel.  They are launched normally.)
+    st = topk_impl(p, batch, 1, scores, ld, max_blocks, q_pos, sel, stream, false);
     if (st) return st;
-    return sparse_mqa_attn(p, batch, 1, q, kv, kv_scales, max_blocks, sel, raw, n_raw, raw_pos0,
-                           q_pos, sinks, out, ws_attn, ws_attn_bytes, stream);
+    return sparse_attn_impl(p, batch, 1, q, kv, kv_scales, max_blocks, sel, raw, n_raw, raw_pos0,
+                            q_pos, sinks, out, ws_attn, ws_attn_bytes, stream, false);
     (void)s;
 }
 

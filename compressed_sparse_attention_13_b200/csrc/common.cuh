@@ -21,6 +21,15 @@ extern __device__ unsigned int g_status;
 
 __device__ __forceinline__ void flag_status(unsigned int bits) { atomicOr(&g_status, bits); }
 
+// Programmatic dependent launch: a kernel launched with it may start before the
+// previous kernel of the stream has finished; pdl_wait() blocks until that
+// kernel has completed and its memory is visible (a no-op without it), and
+// pdl_launch_dependents() lets the next such kernel be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- formats
 // E4M3 code -> float, exact (the hardware conversion to f16 is exact for
 // every E4M3 value, and f16 -> f32 is exact).
@@ -106,6 +115,26 @@ __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { ret
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device): the
 // attribute call is host work that would otherwise sit between launches.
 cudaError_t ensure_smem_impl(const void* kernel, size_t bytes);
+
+// Launch with cudaLaunchKernelEx, optionally as a programmatic dependent of
+// the previous kernel in the stream (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                      bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    if (pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 template <typename K>
 inline cudaError_t ensure_smem(K* kernel, size_t bytes) {
     return ensure_smem_impl(reinterpret_cast<const void*>(kernel), bytes);

@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(128) combine_kernel(int H, int D, int n_splits
                                                       const float* __restrict__ sinks, void* out) {
     __shared__ float wgt[64];
     __shared__ float inv_s;
+    pdl_wait();  // the partials come from the attention kernel before it
     const int64_t row = blockIdx.x;
     const int h = blockIdx.y;
     const float2* ml = part_ml + row * n_splits * H + h;
@@ -257,13 +258,16 @@ __global__ void __launch_bounds__(128) combine_kernel(int H, int D, int n_splits
 }
 
 cudaError_t launch_combine(int act, int H, int D, int n_splits, int64_t rows, const float* part_o,
-                           const float2* part_ml, const float* sinks, void* out, cudaStream_t s) {
+                           const float2* part_ml, const float* sinks, void* out, cudaStream_t s,
+                           bool pdl) {
     if (rows == 0) return cudaSuccess;
     const dim3 grid{unsigned(rows), unsigned(H)};
     if (act == CSA_F32)
-        combine_kernel<CSA_F32><<<grid, 128, 0, s>>>(H, D, n_splits, part_o, part_ml, sinks, out);
+        return launch_ex(combine_kernel<CSA_F32>, grid, dim3(128), 0, s, pdl, H, D, n_splits, part_o,
+                         part_ml, sinks, out);
     else
-        combine_kernel<CSA_BF16><<<grid, 128, 0, s>>>(H, D, n_splits, part_o, part_ml, sinks, out);
+        return launch_ex(combine_kernel<CSA_BF16>, grid, dim3(128), 0, s, pdl, H, D, n_splits, part_o,
+                         part_ml, sinks, out);
     return cudaGetLastError();
 }
 

@@ -138,10 +138,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.raw_full[i], 2);  // expect_tx arrival + arrival after the ids / scales
-            mbar_init(&S.kv_full[i], kConvThreads);
+            mbar_init(&S.kv_full[i], kConvWarps);  // one arrival per converter warp
             mbar_init(&S.kv_empty[i], 1);
             mbar_init(&S.s_full[i], 1);
-            mbar_init(&S.p_full[i], 128);
+            mbar_init(&S.p_full[i], 4);            // one arrival per softmax warp
         }
         mbar_init(&S.o_done, 1);
         mbar_init(&S.q_full, 1);
@@ -149,6 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_mbar_init();
     }
     if (warp == kMmaWarp) { tmem_alloc(&S.tmem_base, 512); tmem_relinquish(); }
+    pdl_launch_dependents();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -211,7 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             fence_proxy_async_smem();
-            mbar_arrive(&S.kv_full[kb]);
+            __syncwarp();  // the whole warp's tile writes are done: one arrival per warp
+            if (lane == 0) mbar_arrive(&S.kv_full[kb]);
         }
     } else if (warp == kIssuerWarp) {
         // ------------------------------------------------------------- issuer
@@ -225,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int blk = 0; blk < 8; ++blk)
                     tma_load_2d(S.q[blk], &map_q, 64 * blk, int32_t(row * kH), &S.q_full);
             }
+            pdl_wait();  // the selected ids come from the kernel before this one
             bool ok = true;
             int issued = 0;
             // software pipeline: the ids of tile lt+1 are loaded during tile lt,
@@ -403,6 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
         int32_t nj0 = 0, nj1 = 0;
+        pdl_wait();  // the selected ids come from the kernel before this one
         if (n_tiles > 0) load_ids(0, nj0, nj1);
         for (int tile = 0; tile < n_tiles; ++tile) {
             const int kb = tile & 1;
@@ -482,7 +486,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (threadIdx.x == 0) S.rescale = 0;
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&S.p_full[kb]);
+            __syncwarp();  // one arrival per warp once all its P writes and O updates are done
+            if (lane == 0) mbar_arrive(&S.p_full[kb]);
         }
         // ----------------------------------------------------------- epilogue
         if (head_lane) {
@@ -635,7 +640,7 @@ static bool cluster_fits(const cudaLaunchConfig_t& cfg) {
     return known[dev][n] == 1;
 }
 
-cudaError_t launch_attn_tc(const AttnArgs& a_in, int64_t rows, cudaStream_t s, bool* combined) {
+cudaError_t launch_attn_tc(const AttnArgs& a_in, int64_t rows, cudaStream_t s, bool* combined, bool pdl) {
     *combined = false;
     if (rows == 0) return cudaSuccess;
     AttnArgs a = a_in;
@@ -667,11 +672,13 @@ cudaError_t launch_attn_tc(const AttnArgs& a_in, int64_t rows, cudaStream_t s, b
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = sm;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = unsigned(a.n_splits);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     // The splits of a row combine inside the kernel when they fit one portable
     // cluster and such clusters can be scheduled; otherwise launch_combine runs.
     if (a.n_splits >= 2 && a.n_splits <= 8) {
@@ -679,14 +686,15 @@ cudaError_t launch_attn_tc(const AttnArgs& a_in, int64_t rows, cudaStream_t s, b
         cfg.numAttrs = 1;
         if (cluster_fits(cfg)) {
             a.fused_combine = 1;
+            cfg.numAttrs = pdl ? 2 : 1;
             e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, map_q, map_win, a);
             if (e == cudaSuccess) *combined = true;
             return e;
         }
-        cfg.attrs = nullptr;
-        cfg.numAttrs = 0;
     }
     a.fused_combine = 0;
+    cfg.attrs = pdl ? &attr[1] : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, attn_tc_kernel, map_q, map_win, a);
 }
 

@@ -16,12 +16,13 @@
 // lane j owns key j's 64 head scores and reduces them without cross-thread
 // traffic.
 //
-// Work is split into 256-key steps (two MMA tiles): the single threads that
-// issue copies and MMAs pay a fixed cost per step in barrier and tcgen05
-// instruction latency, so each step carries two tiles of work.  Persistent
-// CTAs take contiguous ranges of (query row, 256-key step) units and walk them
-// in order, skipping steps past the row's eligible blocks; the k-th eligible
-// step of a CTA is "step it = k".  Warp roles:
+// The single threads that issue copies and MMAs pay a fixed cost per pipeline
+// step in barrier and tcgen05 instruction latency (about 0.5 us), which paces
+// a pipeline; so each SM runs two independent pipelines (two CTAs of 320
+// threads, 256 TMEM columns and ~86 KB of shared memory each).  Persistent
+// CTAs take contiguous ranges of (query row, 128-key step) units and walk
+// them in order, skipping steps past the row's eligible blocks; the k-th
+// eligible step of a CTA is "step it = k".  Warp roles:
 //   warp 0      tensor copy of the step's keys (+ a bulk copy of their scale
 //               bytes) into a kStages ring, and of the query block of each
 //               new row into a kQBufs ring (one elected lane); TMEM allocation
@@ -29,8 +30,8 @@
 //   warps 2-5   scale writers: per step, copy the keys' E8M0 bytes from shared
 //               memory into the TMEM scale-factor layout (and the query's on a
 //               row change) with tcgen05.st
-//   warps 6-13  two epilogue groups; group g owns accumulator g and the steps
-//               with it % 2 == g: ReLU, weights, sum over heads
+//   warps 6-9   epilogue: accumulator it % kAccBufs of step it from TMEM,
+//               ReLU, weights, sum over heads
 // Buffer reuse: the key scales of step it live in TMEM buffer it % kStages,
 // rewritten only after the producer has reused the shared-memory stage, i.e.
 // after the MMA of step it - kStages completed; a row's query scales use
@@ -49,18 +50,22 @@ namespace {
 
 constexpr int kHI = 64, kDI = 128;
 constexpr int kTileKeys = 128;                         // keys per MMA (M)
-constexpr int kStepKeys = 256;                         // keys per pipeline step
+constexpr int kStepKeys = 128;                         // keys per pipeline step
+constexpr int kTilesPerStep = kStepKeys / kTileKeys;
 constexpr int kStages = 8;
 constexpr int kQBufs = 4, kAccBufs = 2;
+constexpr int kEpiGroups = 1;                          // epilogue groups of 4 warps
+constexpr int kCtasPerSm = 2;                          // two independent pipelines per SM
 constexpr int kKeyBytes = kDI / 2;                     // 64: packed E2M1
-constexpr int kAData = kStepKeys * kKeyBytes;          // 16384
+constexpr int kAData = kStepKeys * kKeyBytes;          // 8192
 constexpr int kQData = kHI * kKeyBytes;                // 4096
-constexpr int kAccCols = 2 * 64;                       // two tiles x 64 heads
-constexpr int kSfaCol = kAccBufs * kAccCols;           // 256: 16 columns per stage
-constexpr int kSfbCol = kSfaCol + 16 * kStages;        // 384: 4 columns per buffer
-constexpr int kTmemCols = 512;
-constexpr int kThreads = 448;
+constexpr int kAccCols = kTilesPerStep * 64;           // tiles x 64 heads
+constexpr int kSfaPerStage = 8 * kTilesPerStep;        // two MMA k-steps x 4 columns per tile
+constexpr int kSfaCol = kAccBufs * kAccCols;           // 128
+constexpr int kSfbCol = kSfaCol + kSfaPerStage * kStages;  // 192: 4 columns per buffer
+constexpr int kTmemCols = 256;
 constexpr int kEpiWarp0 = 6;
+constexpr int kThreads = 32 * (kEpiWarp0 + 4 * kEpiGroups);
 static_assert(kSfbCol + 4 * kStages <= kTmemCols, "TMEM columns");
 
 struct IdxTcArgs {
@@ -78,7 +83,7 @@ struct Smem {
     uint8_t a[kStages][kAData];        // 1024-aligned: key steps (64-byte swizzle)
     uint8_t q[kQBufs][kQData];         // query blocks (64-byte swizzle)
     uint32_t a_sf[kStages][kStepKeys]; // keys' four E8M0 bytes
-    float ew[2][kHI];                  // per epilogue group: weights of its current row
+    float ew[kEpiGroups][kHI];         // per epilogue group: weights of its current row
     uint64_t a_full[kStages], a_empty[kStages], sf_full[kStages];
     uint64_t q_full[kQBufs], q_empty[kQBufs];
     uint64_t acc_full[kAccBufs], acc_empty[kAccBufs];
@@ -130,7 +135,7 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_q, const IdxTcArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -140,10 +145,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&S.a_full[i], 1); mbar_init(&S.a_empty[i], 1); mbar_init(&S.sf_full[i], 128);
+            mbar_init(&S.a_full[i], 1); mbar_init(&S.a_empty[i], 1); mbar_init(&S.sf_full[i], 4);  // one arrival per scale-writer warp
         }
         for (int i = 0; i < kQBufs; ++i) { mbar_init(&S.q_full[i], 1); mbar_init(&S.q_empty[i], 1); }
-        for (int i = 0; i < kAccBufs; ++i) { mbar_init(&S.acc_full[i], 1); mbar_init(&S.acc_empty[i], 128); }
+        for (int i = 0; i < kAccBufs; ++i) { mbar_init(&S.acc_full[i], 1); mbar_init(&S.acc_empty[i], 4); }
         fence_mbar_init();
     }
     if (warp == 0) { tmem_alloc(&S.tmem_base, kTmemCols); tmem_relinquish(); }
@@ -213,18 +218,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++rc;
                     ok = mbar_wait(&S.q_full[rc & (kQBufs - 1)], uint32_t(rc / kQBufs) & 1u);
                 }
-                const int b = it & 1;
-                const uint32_t par = uint32_t(it >> 1) & 1u;
+                const int b = it % kAccBufs;
+                const uint32_t par = uint32_t(it / kAccBufs) & 1u;
                 if (ok) ok = mbar_wait(&S.a_full[st], ph);
                 if (ok) ok = mbar_wait(&S.sf_full[st], ph);
                 if (ok && it >= kAccBufs) ok = mbar_wait(&S.acc_empty[b], par ^ 1u);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(S.a[st]), b0 = smem_u32(S.q[rc & (kQBufs - 1)]);
-                const uint32_t sfa = tmem + kSfaCol + 16 * st;
+                const uint32_t sfa = tmem + kSfaCol + kSfaPerStage * st;
                 const uint32_t sfb = tmem + kSfbCol + 4 * (rc & (kStages - 1));
 #pragma unroll
-                for (int t = 0; t < 2; ++t)
+                for (int t = 0; t < kTilesPerStep; ++t)
 #pragma unroll
                     for (int k = 0; k < 2; ++k)
                         mma_mxf4(tmem + b * kAccCols + 64 * t,
@@ -256,16 +261,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             // so this stage's TMEM scale buffer is free
             ok = mbar_wait(&S.a_full[st], ph);
             if (!ok) break;
-            float v[16];
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
+            for (int t = 0; t < kTilesPerStep; ++t) {
+                uint32_t v[8];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const uint32_t wd = S.a_sf[st][128 * t + 32 * c + lane];
-                    v[8 * t + c] = __uint_as_float(wd & 0xFFFFu);
-                    v[8 * t + 4 + c] = __uint_as_float(wd >> 16);
+                    v[c] = wd & 0xFFFFu;
+                    v[4 + c] = wd >> 16;
                 }
-            tmem_st16(tmem + lane_addr + kSfaCol + 16 * st, v);
+                tmem_st8(tmem + lane_addr + kSfaCol + kSfaPerStage * st + 8 * t, v);
+            }
             if (first_of_row) {
                 const uint32_t* qs = reinterpret_cast<const uint32_t*>(a.qIs) + cur_row * kHI;
                 const uint32_t w0 = qs[lane], w1 = qs[32 + lane];
@@ -274,12 +280,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&S.sf_full[st]);
+            __syncwarp();  // the whole warp's stores are done: one arrival per warp
+            if (lane == 0) mbar_arrive(&S.sf_full[st]);
             if (++st == kStages) { st = 0; ph ^= 1u; }
         }
     } else {
         // ----------------------------------------------------------- epilogue
-        const int g = (warp - kEpiWarp0) >> 2;        // group: steps with it % 2 == g
+        const int g = (warp - kEpiWarp0) >> 2;        // group: steps with it % kEpiGroups == g
         const int sub = warp & 3;                     // TMEM lane quarter of this warp
         const int et = threadIdx.x - 32 * (kEpiWarp0 + 4 * g);  // 0..127
         float* ew = S.ew[g];
@@ -287,20 +294,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         int64_t cur_row = -1;
         bool ok = true;
         for (int it = 0; tw.next(a); ++it) {
-            if ((it & 1) != g) continue;
+            if (it % kEpiGroups != g) continue;
             if (tw.row != cur_row) {  // every thread of the group takes this branch together
                 cur_row = tw.row;
                 named_bar(2 + g, 128);
                 if (et < kHI) ew[et] = a.w[cur_row * kHI + et];
                 named_bar(2 + g, 128);
             }
-            if (ok) ok = mbar_wait(&S.acc_full[g], uint32_t(it >> 1) & 1u);
+            const int b = it % kAccBufs;
+            if (ok) ok = mbar_wait(&S.acc_full[b], uint32_t(it / kAccBufs) & 1u);
             if (!ok) continue;
             tc_fence_after();
-            float res[2];
+            float res[kTilesPerStep];
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const uint32_t base = tmem + (uint32_t(sub * 32) << 16) + g * kAccCols + 64 * t;
+            for (int t = 0; t < kTilesPerStep; ++t) {
+                const uint32_t base = tmem + (uint32_t(sub * 32) << 16) + b * kAccCols + 64 * t;
                 // two interleaved partial sums, packed fma over (even, odd)
                 // heads; the 64 head columns are read in two halves
                 uint64_t acc2 = 0;
@@ -310,9 +318,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld16(base + 32 * hf, v[0]);
                     tmem_ld16(base + 32 * hf + 16, v[1]);
                     tmem_wait_ld();
-                    if (t == 1 && hf == 1) {
+                    if (t == kTilesPerStep - 1 && hf == 1) {
                         tc_fence_before();
-                        mbar_arrive(&S.acc_empty[g]);
+                        __syncwarp();  // one arrival per warp once all its loads are done
+                        if (lane == 0) mbar_arrive(&S.acc_empty[b]);
                     }
 #pragma unroll
                     for (int h = 0; h < 32; h += 4) {
@@ -328,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 res[t] = accs.x + accs.y;
             }
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
+            for (int t = 0; t < kTilesPerStep; ++t) {
                 const int64_t j = tw.k0() + kTileKeys * t + sub * 32 + lane;
                 if (j < tw.ne) a.scores[cur_row * a.ld + j] = res[t];
             }
@@ -379,7 +388,7 @@ cudaError_t launch_indexer_tc(const void* qI, const void* qI_s, const float* w, 
     const size_t sm = sizeof(Smem) + 1024;
     cudaError_t e = ensure_smem(indexer_tc_kernel, size_t(sm));
     if (e != cudaSuccess) return e;
-    const int grid = int(std::min<int64_t>(kNumSMs, a.units));
+    const int grid = int(std::min<int64_t>(int64_t(kCtasPerSm) * kNumSMs, a.units));
     indexer_tc_kernel<<<grid, kThreads, sm, s>>>(map_k, map_q, a);
     return cudaGetLastError();
 }

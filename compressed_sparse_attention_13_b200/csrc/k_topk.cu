@@ -100,6 +100,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(
     __shared__ int hist[2048];
     __shared__ int2 warp_tot[32];
     __shared__ int found_digit, found_above;
+    pdl_wait();  // the scores come from the kernel before this one
+    pdl_launch_dependents();
     const int tid = threadIdx.x;
     const int64_t row = blockIdx.x;
     const float* s = scores + row * ld;
@@ -161,6 +163,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_smem_kernel(
     __shared__ int whist[32][256];
     __shared__ int2 warp_tot[32];
     __shared__ int found_digit, found_above;
+    pdl_wait();  // the scores come from the kernel before this one
+    pdl_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t row = blockIdx.x;
     const float* s = scores + row * ld;
@@ -272,6 +276,8 @@ __global__ void __cluster_dims__(kClu, 1, 1) __launch_bounds__(kCluThreads)
     __shared__ int2 cta_tot;
     __shared__ int found_digit, found_above;
     cg::cluster_group cluster = cg::this_cluster();
+    pdl_wait();  // the scores come from the kernel before this one
+    pdl_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int r = int(cluster.block_rank());
     const int64_t row = blockIdx.x / kClu;
@@ -387,34 +393,33 @@ __global__ void __cluster_dims__(kClu, 1, 1) __launch_bounds__(kCluThreads)
 template <int E>
 static cudaError_t launch_topk_cluster(const float* scores, int64_t ld, int64_t max_blocks,
                                        const int64_t* q_pos, int m, int W, int k, int64_t rows,
-                                       int32_t* idx, cudaStream_t s) {
-    topk_cluster_kernel<E><<<unsigned(rows * kClu), kCluThreads, 0, s>>>(scores, ld, max_blocks,
-                                                                        q_pos, m, W, k, idx);
-    return cudaGetLastError();
+                                       int32_t* idx, cudaStream_t s, bool pdl) {
+    return launch_ex(topk_cluster_kernel<E>, dim3(unsigned(rows * kClu)), dim3(kCluThreads), 0, s, pdl,
+                     scores, ld, max_blocks, q_pos, m, W, k, idx);
 }
 
 cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, const int64_t* q_pos,
-                        int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s) {
+                        int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s, bool pdl) {
     if (rows == 0) return cudaSuccess;
     // Few rows cannot fill the GPU with one CTA each: give each row a cluster.
     if (rows <= 2 * kNumSMs / kClu && k <= kClu * kCluThreads && max_blocks <= kClu * kCluThreads * 72) {
         const int64_t per = ceil_div(max_blocks, kClu * kCluThreads);
-        if (per <= 2) return launch_topk_cluster<2>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
-        if (per <= 4) return launch_topk_cluster<4>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
-        if (per <= 8) return launch_topk_cluster<8>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
-        if (per <= 16) return launch_topk_cluster<16>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
-        if (per <= 32) return launch_topk_cluster<32>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
-        return launch_topk_cluster<72>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s);
+        if (per <= 2) return launch_topk_cluster<2>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
+        if (per <= 4) return launch_topk_cluster<4>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
+        if (per <= 8) return launch_topk_cluster<8>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
+        if (per <= 16) return launch_topk_cluster<16>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
+        if (per <= 32) return launch_topk_cluster<32>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
+        return launch_topk_cluster<72>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
     }
     if (max_blocks <= kTopkSmemMax) {
         const size_t sm = size_t(std::max<int64_t>(max_blocks, 1)) * 4;
         cudaError_t e = ensure_smem(topk_smem_kernel, size_t(sm));
         if (e != cudaSuccess) return e;
-        topk_smem_kernel<<<unsigned(rows), kTopkThreads, sm, s>>>(scores, ld, max_blocks, q_pos, m, W, k, idx);
-    } else {
-        topk_kernel<<<unsigned(rows), kTopkThreads, 0, s>>>(scores, ld, max_blocks, q_pos, m, W, k, idx);
+        return launch_ex(topk_smem_kernel, dim3(unsigned(rows)), dim3(kTopkThreads), sm, s, pdl, scores, ld,
+                         max_blocks, q_pos, m, W, k, idx);
     }
-    return cudaGetLastError();
+    return launch_ex(topk_kernel, dim3(unsigned(rows)), dim3(kTopkThreads), 0, s, pdl, scores, ld,
+                     max_blocks, q_pos, m, W, k, idx);
 }
 
 }  // namespace csa

@@ -42,16 +42,23 @@ cudaError_t launch_indexer_tc(const void* qI, const void* qI_s, const float* w, 
                               const void* kI_s, int64_t max_blocks, const int64_t* q_pos,
                               int batch, int n_q, int m, int W, float* scores, int64_t ld,
                               cudaStream_t s);
+// pdl: launched as a programmatic dependent of the previous kernel (which
+// wrote `scores`); only set when that kernel is known.
 cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, const int64_t* q_pos,
-                        int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s);
+                        int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s,
+                        bool pdl = false);
 bool attn_tc_supported(int act, int kvf, int H, int D);
 bool attn_tc_rows_fit(int64_t max_entries, int64_t n_raw);
 // Sets *combined when the splits were combined inside the kernel (no
 // launch_combine needed).
-cudaError_t launch_attn_tc(const AttnArgs& a, int64_t rows, cudaStream_t s, bool* combined);
+// pdl: launched as a programmatic dependent of the kernel that wrote a.idx
+// (the query, entries and window are read before waiting for it).
+cudaError_t launch_attn_tc(const AttnArgs& a, int64_t rows, cudaStream_t s, bool* combined,
+                           bool pdl = false);
 cudaError_t launch_attn_simt(int act, int kvf, const AttnArgs& a, int64_t rows, cudaStream_t s);
 bool attn_simt_supported(int act, int kvf, int H, int D);
 cudaError_t launch_combine(int act, int H, int D, int n_splits, int64_t rows, const float* part_o,
-                           const float2* part_ml, const float* sinks, void* out, cudaStream_t s);
+                           const float2* part_ml, const float* sinks, void* out, cudaStream_t s,
+                           bool pdl = false);
 
 }  // namespace csa
