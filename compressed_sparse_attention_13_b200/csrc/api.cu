@@ -108,7 +108,7 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
     AttnArgs a;
     a.H = p->n_heads; a.D = p->head_dim; a.m = p->m; a.W = p->window; a.k = p->top_k;
     a.scale = p->scale;
-    a.q = q; a.kv = kv; a.kv_s = kv_s; a.max_entries = max_entries; a.idx = idx;
+    a.q = q; a.kv = kv; a.kv_s = kv_s; a.kv_fmt = p->kv_fmt; a.max_entries = max_entries; a.idx = idx;
     a.raw = raw; a.n_raw = n_raw; a.raw_pos0 = raw_pos0; a.q_pos = q_pos; a.sinks = sinks;
     a.n_q = n_q; a.n_splits = plan.n_splits; a.out = out;
     a.part_o = (float*)ws;
@@ -116,6 +116,7 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
     const bool tc = attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim) &&
                     attn_tc_rows_fit(max_entries, n_raw);
     a.fused_combine = 0;
+    a.row_base = 0;
     bool combined = false;
     int st = cuda_status(tc ? launch_attn_tc(a, rows, s, &combined, pdl)
                             : launch_attn_simt(p->act_fmt, p->kv_fmt, a, rows, s));
@@ -205,6 +206,9 @@ int indexer_score(const csa_params* p, int32_t batch, int32_t n_q, const void* q
         return cuda_status(launch_indexer_tc(qI, qI_scales, w, kI, kI_scales, max_blocks, q_pos,
                                              batch, n_q, p->m, p->window, scores, ld_scores,
                                              (cudaStream_t)stream));
+    if (indexer_bf16_tc_supported(p->idx_fmt, p->idx_heads, p->idx_dim, max_blocks, batch, n_q))
+        return cuda_status(launch_indexer_bf16_tc(qI, w, kI, max_blocks, q_pos, batch, n_q, p->m,
+                                                  p->window, scores, ld_scores, (cudaStream_t)stream));
     return cuda_status(launch_indexer_simt(p->idx_fmt, p->idx_heads, p->idx_dim, p->m, p->window,
                                            qI, qI_scales, w, kI, kI_scales, max_blocks, q_pos,
                                            batch, n_q, max_blocks, scores, ld_scores,

@@ -25,11 +25,16 @@
 //
 // Data movement: the query (8 tensor copies) and window tiles (8 tensor
 // copies from a [batch][n_raw][512] map; rows past the sequence read as
-// zero) land directly in operand layout.  A pooled tile's FP8 rows land by
-// bulk copy (one per selected row, or one per tile for dense HCA rows) in the
-// upper half of the tile's own buffer and are dequantised in place: dims
-// 0..255 go to the lower half, dims 256..511 are read into registers before
-// any thread overwrites the upper half.
+// zero) land directly in operand layout.  Pooled entries come in two stored
+// formats (template parameter KVF):
+//  * FP8: a tile's rows land by bulk copy (one per selected row, or one per
+//    tile for dense HCA rows) in the upper half of the tile's own buffer and
+//    are dequantised in place: dims 0..255 go to the lower half, dims
+//    256..511 are read into registers before any thread overwrites the upper
+//    half.
+//  * bf16: selected rows are gathered by the converter warps with 16-byte
+//    asynchronous copies straight to their swizzled place (unselected slots
+//    are zero-filled); dense HCA tiles arrive by tensor copy like the window.
 //
 // Roles (448 threads): warps 0-3 softmax (lanes 0-15: one head each) and
 // epilogue (all 128 lanes: one dim each per quarter), warps 4-11 convert,
@@ -70,6 +75,7 @@ struct SmemAttn {
     uint8_t p[2][kH * 128];         // 2 buffers x [64 heads][64 items bf16] (16 KB)
     float kvs[2][kTile][kD / 64];   // per buffer: FP8 scales of the tile's items (4 KB)
     int32_t valid[2][kTile];        // per buffer: item holds data
+    int32_t ids[2][kTile];          // per buffer: entry id of each item (bf16 gather), -1 if none
     float alpha[kH], fin[kH];
     float2 ml[kH];                  // cluster combine: this split's (max in log2 units, sum) per head
     float cw[8][kH], cinv[kH];      // cluster combine: weight of each split, 1 / denominator
@@ -105,6 +111,18 @@ __device__ __forceinline__ uint4 dequant8(uint2 w, float s) {
                       bf16x2_scaled(f3, s));
 }
 
+// 16-byte global -> shared copy that bypasses L1; fewer than 16 source bytes
+// (here 0) zero-fill the destination
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sm100::smem_u32(dst)), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -113,15 +131,18 @@ __device__ __forceinline__ float ex2(float x) {
 
 }  // namespace
 
+template <int KVF>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_win,
-                   const AttnArgs a) {
+                   const __grid_constant__ CUtensorMap map_kv, const AttnArgs a) {
+    static_assert(KVF == CSA_FP8_S64 || KVF == CSA_BF16, "pooled entries are FP8 or bf16");
+    constexpr bool kFp8 = KVF == CSA_FP8_S64;
     extern __shared__ uint8_t smem_raw[];
     SmemAttn& S = *reinterpret_cast<SmemAttn*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     using namespace sm100;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    const int64_t row = blockIdx.y;
+    const int64_t row = a.row_base + blockIdx.y;
     const int split = blockIdx.x;
     const int64_t b = row / a.n_q;
     const int64_t t = a.q_pos[row];
@@ -167,7 +188,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kb = lt & 1;
             ok = mbar_wait(&S.raw_full[kb], uint32_t((lt >> 1) & 1));
             if (!ok) break;
-            if (tile0 + lt < kv_tiles) {
+            if (!kFp8 && a.idx && tile0 + lt < kv_tiles) {
+                // bf16 gather: 64 threads per 1024-byte row (one 16-byte
+                // granule each), four rows per pass
+                const uint8_t* kv_seq = (const uint8_t*)a.kv + b * a.max_entries * int64_t(kD * 2);
+                const int g = pt & 63;
+#pragma unroll
+                for (int u = 0; u < kTile / 4; ++u) {
+                    const int item = (pt >> 6) + 4 * u;
+                    const int32_t id = S.ids[kb][item];
+                    const uint8_t* src = kv_seq + int64_t(id < 0 ? 0 : id) * (kD * 2) + 16 * g;
+                    cp_async16(S.kv[kb][g >> 3] + sw128_offset(item, g & 7), src, id < 0 ? 0u : 16u);
+                }
+                cp_async_wait_all();
+            } else if (kFp8 && tile0 + lt < kv_tiles) {
                 const uint8_t* raw = S.kv[kb][kRawBlk];  // [64 items][512 E4M3] over blocks 4..7
                 // dims 0..255 -> lower half (the rows sit in the upper half)
 #pragma unroll
@@ -204,7 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             dequant8(w[qt][u], sc[qt][u]);
                     }
             } else {
-                // window tile: already in place; clear rows past the window
+                // window tile (or dense bf16 tile): already in place; clear
+                // rows past the window or past the eligible entries
                 for (int i = pt; i < kTile * 8 * 8; i += kConvThreads) {
                     const int item = i >> 6, blk = (i >> 3) & 7, ch = i & 7;
                     if (!S.valid[kb][item])
@@ -219,8 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------- issuer
         // lane l handles items l and l + 32 of each tile
         if (n_tiles > 0) {
-            const uint8_t* kv_seq = (const uint8_t*)a.kv + b * a.max_entries * int64_t(kD);
-            const float* kvs_seq = (const float*)a.kv_s + b * a.max_entries * int64_t(kD / 64);
+            const uint8_t* kv_seq = (const uint8_t*)a.kv + b * a.max_entries * int64_t(kFp8 ? kD : 0);
+            const float* kvs_seq = (const float*)a.kv_s + b * a.max_entries * int64_t(kFp8 ? kD / 64 : 0);
             if (lane == 0) {
                 mbar_arrive_expect_tx(&S.q_full, uint32_t(kH * kD * 2));
 #pragma unroll
@@ -255,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (pooled && slot < n_kv && j >= a.max_entries) flag_status(CSA_DEV_BAD_INDEX);
                     sr[h2] = (pooled && slot < n_kv && j >= 0 && j < a.max_entries) ? int32_t(j) : -1;
                     scl[h2][0] = scl[h2][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (a.idx && sr[h2] >= 0) {
+                    if (kFp8 && a.idx && sr[h2] >= 0) {
                         const float4* sp = reinterpret_cast<const float4*>(kvs_seq + int64_t(sr[h2]) * (kD / 64));
                         scl[h2][0] = sp[0];
                         scl[h2][1] = sp[1];
@@ -264,7 +299,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lt + 1 < n_tiles) load_ids(lt + 1, jn);
                 if (lt >= 2) ok = mbar_wait(&S.kv_empty[kb], uint32_t(((lt >> 1) - 1) & 1));
                 if (!ok) break;
-                if (pooled) {
+                if (pooled && !kFp8) {
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        S.valid[kb][lane + 32 * h2] = sr[h2] >= 0;
+                        S.ids[kb][lane + 32 * h2] = sr[h2];
+                    }
+                    if (!a.idx) {
+                        // dense: the tile's rows are consecutive; rows past the
+                        // entries read as zero, rows past n_kv are cleared
+                        const int64_t j0 = int64_t(T) * kTile;
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&S.raw_full[kb], uint32_t(kTile * kD * 2));
+#pragma unroll
+                            for (int blk = 0; blk < 8; ++blk)
+                                tma_load_3d(S.kv[kb][blk], &map_kv, 64 * blk, int32_t(j0), int32_t(b),
+                                            &S.raw_full[kb]);
+                        }
+                    } else if (lane == 0) {
+                        mbar_arrive(&S.raw_full[kb]);  // the converters gather the rows
+                    }
+                } else if (pooled) {
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) S.valid[kb][lane + 32 * h2] = sr[h2] >= 0;
                     uint8_t* dst = S.kv[kb][kRawBlk];
@@ -614,7 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 bool attn_tc_supported(int act, int kvf, int H, int D) {
-    return act == CSA_BF16 && kvf == CSA_FP8_S64 && H == kH && D == kD;
+    return act == CSA_BF16 && (kvf == CSA_FP8_S64 || kvf == CSA_BF16) && H == kH && D == kD;
 }
 
 bool attn_tc_rows_fit(int64_t max_entries, int64_t n_raw) {
@@ -622,7 +677,8 @@ bool attn_tc_rows_fit(int64_t max_entries, int64_t n_raw) {
 }
 
 // Whether clusters of cfg's size can be scheduled for this kernel on the
-// current device (queried once per device and size).
+// current device (queried once per device, entry format and size).
+template <int KVF>
 static bool cluster_fits(const cudaLaunchConfig_t& cfg) {
     static std::mutex mu;
     static int known[64][9];  // 0 unknown, 1 yes, 2 no
@@ -632,7 +688,7 @@ static bool cluster_fits(const cudaLaunchConfig_t& cfg) {
     std::lock_guard<std::mutex> lock(mu);
     if (known[dev][n] == 0) {
         int n_clusters = 0;
-        const bool ok = cudaOccupancyMaxActiveClusters(&n_clusters, attn_tc_kernel, &cfg) == cudaSuccess &&
+        const bool ok = cudaOccupancyMaxActiveClusters(&n_clusters, attn_tc_kernel<KVF>, &cfg) == cudaSuccess &&
                         n_clusters > 0;
         if (!ok) (void)cudaGetLastError();
         known[dev][n] = ok ? 1 : 2;
@@ -640,10 +696,8 @@ static bool cluster_fits(const cudaLaunchConfig_t& cfg) {
     return known[dev][n] == 1;
 }
 
-cudaError_t launch_attn_tc(const AttnArgs& a_in, int64_t rows, cudaStream_t s, bool* combined, bool pdl) {
-    *combined = false;
-    if (rows == 0) return cudaSuccess;
-    AttnArgs a = a_in;
+template <int KVF>
+static cudaError_t launch_attn_tc_fmt(AttnArgs a, int64_t rows, cudaStream_t s, bool* combined, bool pdl) {
     if (rows * kH >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
     // query [rows * 64][512] bf16 and window tokens [batch][n_raw][512] bf16,
     // both read as [64 rows][64 dims] boxes with 128-byte swizzle
@@ -664,11 +718,23 @@ cudaError_t launch_attn_tc(const AttnArgs& a_in, int64_t rows, cudaStream_t s, b
                              CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
+    // bf16 entries [batch][max_entries][512]: dense tiles read as [64 rows][64 dims] boxes
+    CUtensorMap map_kv;
+    memset(&map_kv, 0, sizeof(map_kv));
+    if (KVF == CSA_BF16 && !a.idx && a.max_entries > 0) {
+        const int64_t batch = rows / a.n_q;
+        const uint64_t kd[3] = {uint64_t(kD), uint64_t(a.max_entries), uint64_t(batch)};
+        const uint64_t ks[2] = {uint64_t(kD) * 2, uint64_t(a.max_entries) * kD * 2};
+        const uint32_t box3[3] = {64, 64, 1};
+        if (!encode_tile_map(&map_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.kv, kd, ks, box3,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
     const size_t sm = sizeof(SmemAttn) + 1024;
-    cudaError_t e = ensure_smem(attn_tc_kernel, sm);
+    cudaError_t e = ensure_smem(attn_tc_kernel<KVF>, sm);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.n_splits, unsigned(rows));
+    cfg.gridDim = dim3(a.n_splits, unsigned(std::min<int64_t>(rows, 65535)));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = sm;
     cfg.stream = s;
@@ -684,10 +750,10 @@ cudaError_t launch_attn_tc(const AttnArgs& a_in, int64_t rows, cudaStream_t s, b
     if (a.n_splits >= 2 && a.n_splits <= 8) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cluster_fits(cfg)) {
+        if (cluster_fits<KVF>(cfg)) {
             a.fused_combine = 1;
             cfg.numAttrs = pdl ? 2 : 1;
-            e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, map_q, map_win, a);
+            e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<KVF>, map_q, map_win, map_kv, a);
             if (e == cudaSuccess) *combined = true;
             return e;
         }
@@ -695,7 +761,23 @@ cudaError_t launch_attn_tc(const AttnArgs& a_in, int64_t rows, cudaStream_t s, b
     a.fused_combine = 0;
     cfg.attrs = pdl ? &attr[1] : nullptr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, attn_tc_kernel, map_q, map_win, a);
+    // the grid's y extent is at most 65535: long prefill chunks take several launches
+    constexpr int64_t kMaxY = 65535;
+    for (int64_t r0 = 0; r0 < rows; r0 += kMaxY) {
+        a.row_base = r0;
+        cfg.gridDim.y = unsigned(std::min(kMaxY, rows - r0));
+        e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<KVF>, map_q, map_win, map_kv, a);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_attn_tc(const AttnArgs& a, int64_t rows, cudaStream_t s, bool* combined, bool pdl) {
+    *combined = false;
+    if (rows == 0) return cudaSuccess;
+    if (a.kv_fmt == CSA_BF16) return launch_attn_tc_fmt<CSA_BF16>(a, rows, s, combined, pdl);
+    if (a.kv_fmt == CSA_FP8_S64) return launch_attn_tc_fmt<CSA_FP8_S64>(a, rows, s, combined, pdl);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace csa

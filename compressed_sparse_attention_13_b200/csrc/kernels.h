@@ -11,6 +11,7 @@ struct AttnArgs {
     const void* q;          // [rows][H][D] act format
     const void* kv;         // [batch][max_entries][D] kv format
     const void* kv_s;       // scales of kv (FP8_S64) or null
+    int kv_fmt;             // stored format of kv
     int64_t max_entries;
     const int32_t* idx;     // [rows][k] selected ids, or null for dense (HCA)
     const void* raw;        // [batch][n_raw][D] act format
@@ -25,6 +26,7 @@ struct AttnArgs {
     float2* part_ml;          // [rows][n_splits][H] (running max, running sum)
     int fused_combine;        // tensor-core kernel: the splits of a row form a cluster and
                               // combine through distributed shared memory (set by the launcher)
+    int64_t row_base;         // tensor-core kernel: first row of this launch (set by the launcher)
 };
 
 cudaError_t launch_compress(int in_fmt, int out_fmt, const void* x, const void* z,
@@ -42,6 +44,10 @@ cudaError_t launch_indexer_tc(const void* qI, const void* qI_s, const float* w, 
                               const void* kI_s, int64_t max_blocks, const int64_t* q_pos,
                               int batch, int n_q, int m, int W, float* scores, int64_t ld,
                               cudaStream_t s);
+bool indexer_bf16_tc_supported(int fmt, int HI, int dI, int64_t max_blocks, int64_t batch, int n_q);
+cudaError_t launch_indexer_bf16_tc(const void* qI, const float* w, const void* kI, int64_t max_blocks,
+                                   const int64_t* q_pos, int batch, int n_q, int m, int W,
+                                   float* scores, int64_t ld, cudaStream_t s);
 // pdl: launched as a programmatic dependent of the previous kernel (which
 // wrote `scores`); only set when that kernel is known.
 cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, const int64_t* q_pos,

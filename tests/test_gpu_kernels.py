@@ -129,6 +129,8 @@ def test_compress_quantised_out(act, m, d, n_blocks, fmt):
 @pytest.mark.parametrize("idx,HI,dI,n_q,nb,m,W", [
     ("f32", 4, 32, 40, 256, 4, 64),
     ("bf16", 64, 128, 12, 700, 4, 128),
+    ("bf16", 64, 128, 13, 300, 4, 128),
+    ("bf16", 64, 128, 2, 300, 4, 128),
     ("mxfp4", 64, 128, 3, 2100, 4, 128),
 ])
 def test_indexer_matches_oracle(idx, HI, dI, n_q, nb, m, W):
@@ -222,6 +224,8 @@ def _attn_case(act, kvf, H, d, batch, n_q, n_ent, W, k, m, seed, scale):
     ("bf16", "fp8", 64, 512, 12, 700, 128, 512, 4),
     ("bf16", "fp8", 64, 512, 20, 400, 128, 256, 4),
     ("bf16", "bf16", 64, 512, 4, 300, 128, 64, 4),
+    ("bf16", "bf16", 64, 512, 3, 700, 128, 512, 4),
+    ("bf16", "bf16", 64, 512, 160, 900, 128, 512, 4),
 ])
 def test_sparse_attention_matches_oracle(act, kvf, H, d, n_q, n_ent, W, k, m):
     batch, seed, scale = 2, 5, 1 / math.sqrt(d)
@@ -254,6 +258,8 @@ def test_sparse_attention_matches_oracle(act, kvf, H, d, n_q, n_ent, W, k, m):
 @pytest.mark.parametrize("act,kvf,H,d,n_q,n_ent,W,m", [
     ("f32", "f32", 8, 64, 10, 300, 64, 4),
     ("bf16", "fp8", 64, 512, 2, 1500, 128, 128),
+    ("bf16", "bf16", 64, 512, 2, 1500, 128, 128),
+    ("bf16", "bf16", 64, 512, 3, 333, 128, 4),
 ])
 def test_hca_attention_matches_oracle(act, kvf, H, d, n_q, n_ent, W, m):
     batch, seed, scale = 2, 6, 1 / math.sqrt(d)
