@@ -232,6 +232,14 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     K.lib()
     hbm_peak, bf16_peak, peak_kind = peaks()
+    if args.only_legs:
+        # one GPU, the named extra legs alone (a small command to profile them)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        legs = {"hca": lambda: bench_hca(args, dev, flush, stream, hbm_peak),
+                "prefill": lambda: bench_prefill(dev, flush, stream, bf16_peak),
+                "stack": lambda: bench_stack(dev, flush, stream, hbm_peak)}
+        print(json.dumps({n: legs[n]() for n in args.only_legs.split(",")}), flush=True)
+        return
 
     w = WORKLOADS[WORKLOAD]
     S = setup_csa_decode(w, dev)
@@ -315,15 +323,20 @@ def run_ours(args):
         "step_gbs": round(by["step"] / (t_ms / args.steps / 1e3) / 1e9, 1),
         "e2e": {"value": round(e2e_value, 1), "unit": "tok/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * args.steps,
+        # indexer, top-k and attention (the split combine runs in the attention's cluster)
+        "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
     }
+    legs = set(args.legs.split(",")) if args.legs else {"hca", "prefill", "stack"}
     if world == 1 and rank == 0 and not args.no_extra:
-        result["hca_decode"] = bench_hca(args, dev, flush, stream, hbm_peak)
+        if "hca" in legs:
+            result["hca_decode"] = bench_hca(args, dev, flush, stream, hbm_peak)
         del S
         torch.cuda.empty_cache()
-        for key, leg in (("prefill_8k_bf16", lambda: bench_prefill(dev, flush, stream, bf16_peak)),
-                         ("stack_c4", lambda: bench_stack(dev, flush, stream, hbm_peak))):
+        for key, name, leg in (("prefill_8k_bf16", "prefill", lambda: bench_prefill(dev, flush, stream, bf16_peak)),
+                               ("stack_c4", "stack", lambda: bench_stack(dev, flush, stream, hbm_peak))):
+            if name not in legs:
+                continue
             try:
                 result[key] = leg()
             except Exception as exc:  # an extra leg must not lose the main line
@@ -409,16 +422,34 @@ def bench_prefill(dev, flush, stream, bf16_peak):
     ws = torch.empty(K.csa_workspace_size(p, K.OP_PREFILL, B, T, nb), dtype=torch.uint8, device=dev)
     fn = lambda: K.csa_prefill(p, B, T, 0, t_["x"], T, 0, t_["z"], t_["bias"], t_["q"], qI, t_["w"], kv,
                                kI, nb, t_["sinks"], out, sel, ws)
-    times = time_steps(fn, 3, 3, flush, stream)
+    times = time_steps(fn, 5, 3, flush, stream)
     t = statistics.median(times)
     pi, pa = _causal_pairs(T, m, W, k)
-    flops = B * (pi * 2 * HI * dI + pa * 4 * H * d)
+    f_idx, f_att = B * pi * 2 * HI * dI, B * pa * 4 * H * d
+    flops = f_idx + f_att
     tf = flops / (t / 1e3) / 1e12
+    # the stages alone, on the entries and selections the chunk produced
+    scores = torch.empty(B * T, nb, dtype=torch.float32, device=dev)
+    q_pos = torch.arange(T, dtype=torch.int64, device=dev).repeat(B)
+    pos0 = torch.zeros(B, dtype=torch.int64, device=dev)
+    stages = {
+        "indexer_score": lambda: K.indexer_score(p, B, T, qI, t_["w"], kI, nb, q_pos, scores, nb),
+        "topk_select": lambda: K.topk_select(p, B, T, scores, nb, nb, q_pos, sel),
+        "sparse_mqa_attn": lambda: K.sparse_mqa_attn(p, B, T, t_["q"], kv, nb, sel, t_["x"], T, pos0, q_pos,
+                                                     t_["sinks"], out, ws),
+    }
+    st = {n: statistics.median(time_steps(f, 5, 3, flush, stream)) for n, f in stages.items()}
+    assert K.csa_device_status(reset=True) == 0
+    tf_idx = f_idx / (st["indexer_score"] / 1e3) / 1e12
+    tf_att = f_att / (st["sparse_mqa_attn"] / 1e3) / 1e12
+    roof = lambda kern, a: {"kernel": kern, "bound": "tensor", "achieved": round(a, 2), "peak": bf16_peak,
+                            "unit": "TFLOP/s", "frac": round(a / bf16_peak, 4)}
     return {"workload": "csa_prefill_8k_bf16", "value": round(B * T / (t / 1e3), 1), "unit": "tok/s",
             "ms_per_step": round(t, 3), "flop": flops,
-            "roofline": {"kernel": "csa_prefill (CUDA-core bf16 indexer + attention)", "bound": "tensor",
-                         "achieved": round(tf, 2), "peak": bf16_peak, "unit": "TFLOP/s",
-                         "frac": round(tf / bf16_peak, 4)}}
+            "roofline": roof("csa_prefill (all stages)", tf),
+            "stages_ms": {n: round(v, 4) for n, v in st.items()},
+            "stage_roofline": {"indexer_score": roof("indexer_bf16_tc_kernel", tf_idx),
+                               "sparse_mqa_attn": roof("attn_tc_kernel<1> (bf16 entries)", tf_att)}}
 
 
 def bench_stack(dev, flush, stream, hbm_peak):
@@ -621,7 +652,11 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-extra", action="store_true", help="skip the HCA decode leg")
+    ap.add_argument("--no-extra", action="store_true", help="skip the extra legs")
+    ap.add_argument("--legs", default="", help="extra legs to run, comma-separated among hca, prefill, "
+                    "stack (default: all)")
+    ap.add_argument("--only-legs", default="", help="run only these extra legs (comma-separated among "
+                    "hca, prefill, stack) and print their results, without the main line")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     args = ap.parse_args()

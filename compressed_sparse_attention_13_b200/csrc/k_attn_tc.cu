@@ -487,9 +487,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 al = m_run == -INFINITY ? 0.f : ex2(m_run - mx);
                 m_run = mx;
             }
-            // P.V of the previous tile must be done before P[kb] (read by P.V
-            // two tiles back) is rewritten and before O^T is rescaled
-            if (ok && tile > 0) ok = mbar_wait(&S.o_done, uint32_t((tile - 1) & 1));
+            // P[kb] was read by P.V two tiles back: that one must be done (its
+            // completion also releases the tile buffer, hence kv_empty)
+            if (ok && tile >= 2) ok = mbar_wait(&S.kv_empty[kb], uint32_t(((tile >> 1) - 1) & 1));
             // pass 2: P = exp2(x - m) as bf16 rows of the K-major B tile, and the sum
             float sum = 0.f;
 #pragma unroll 1
@@ -523,6 +523,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             named_bar(1, 128);
             if (ok && S.rescale != 0) {
+                // O^T is rescaled only once P.V of the previous tile is done
+                // (P.V two tiles back is done, so the phase is unambiguous)
+                ok = mbar_wait(&S.o_done, uint32_t((tile - 1) & 1));
                 tc_fence_after();
 #pragma unroll 1
                 for (int qc = 0; qc < 16; ++qc) {  // 16-column chunks of O^T; rolled to keep registers free
@@ -565,6 +568,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         named_bar(1, 128);
+        // every P.V done: the one two tiles back first, so that the last
+        // o_done phase is unambiguous
+        if (n_tiles >= 2 && ok)
+            ok = mbar_wait(&S.kv_empty[(n_tiles - 2) & 1], uint32_t(((n_tiles - 2) >> 1) & 1));
         if (n_tiles > 0 && ok) ok = mbar_wait(&S.o_done, uint32_t((n_tiles - 1) & 1));
         tc_fence_after();
         // Every P.V has completed, so the two tile buffers (128 KB) are free:
