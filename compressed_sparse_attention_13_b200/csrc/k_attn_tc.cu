@@ -383,15 +383,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = mbar_wait(&S.q_full, 0);
             // QK(t) may run at most one tile ahead of P.V: it overwrites S[t&1],
             // which the softmax of tile t-2 has finished reading once P.V(t-2)
-            // has been issued.  Each wait is a single poll; the loop as a whole
-            // is bounded by kWaitNs without progress.
+            // has been issued.  Each wait is a single non-blocking test; the
+            // loop as a whole is bounded by kWaitNs without progress.
             int qk_t = 0, pv_t = 0;
             uint64_t t_last = global_ns();
             while (ok && pv_t < n_tiles) {
                 bool progressed = false;
                 if (qk_t < n_tiles && qk_t <= pv_t + 1) {
                     const int kb = qk_t & 1;
-                    if (mbar_try_wait(&S.kv_full[kb], uint32_t((qk_t >> 1) & 1))) {
+                    if (mbar_test_wait(&S.kv_full[kb], uint32_t((qk_t >> 1) & 1))) {
                         tc_fence_after();
                         const uint32_t kv0 = smem_u32(S.kv[kb][0]);
 #pragma unroll
@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (pv_t < qk_t) {
                     const int kb = pv_t & 1;
-                    if (mbar_try_wait(&S.p_full[kb], uint32_t((pv_t >> 1) & 1))) {
+                    if (mbar_test_wait(&S.p_full[kb], uint32_t((pv_t >> 1) & 1))) {
                         tc_fence_after();
                         const uint32_t kv0 = smem_u32(S.kv[kb][0]), pp = smem_u32(S.p[kb]);
 #pragma unroll
