@@ -161,6 +161,24 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
+def max_over_ranks(value: float, device) -> float:
+    """The largest of every rank's value (all ranks call this, in the same
+    order): a multi-GPU step is as slow as its slowest replica."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(batch: int, steps: int, world: int, t_ms: float) -> float:
+    """Tokens per second of the whole job: every replica decodes `batch`
+    sequences per step, and the job takes the slowest replica's time."""
+    return batch * steps * world / (t_ms / 1e3)
+
+
 def setup_csa_decode(w, dev):
     import torch
 
@@ -298,14 +316,9 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         times = time_steps(step, args.steps, args.warmup, flush, stream)
         barrier()
-    t_ms = sum(times)
-    if world > 1:
-        tt = torch.tensor([t_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_ms = float(tt.item())
+    t_ms = max_over_ranks(sum(times), dev)
     assert K.csa_device_status(reset=True) == 0
-    tokens = w.batch * args.steps * world
-    value = tokens / (t_ms / 1e3)
+    value = job_throughput(w.batch, args.steps, world, t_ms)
 
     # per-kernel times of the decode step (same launch configuration)
     nb = S["nb"]
