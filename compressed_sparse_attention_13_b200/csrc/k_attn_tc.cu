@@ -593,11 +593,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 32; ++i) o[i] = 0.f;
                 }
                 if (final_out) {
+                    // the 32 factors first: loads that followed stores into
+                    // the same shared memory would each wait for the store
+                    float f[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int hh = 32 * hf + i;
-                        so16[hh * kD + dim] = __float2bfloat16_rn(o[i] * S.fin[hh]);
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 f4 = reinterpret_cast<const float4*>(&S.fin[32 * hf])[j];
+                        f[4 * j] = f4.x; f[4 * j + 1] = f4.y; f[4 * j + 2] = f4.z; f[4 * j + 3] = f4.w;
                     }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) so16[(32 * hf + i) * kD + dim] = __float2bfloat16_rn(o[i] * f[i]);
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) so32[(32 * hf + i) * kD + dim] = o[i];
