@@ -59,7 +59,7 @@ static int cuda_status(cudaError_t e) {
 // ------------------------------------------------------------ attention
 static int choose_splits(int64_t rows, int64_t items_per_row) {
     // Enough CTAs to cover every SM about twice, with at least 64 items per split.
-    if (rows >= 2 * kNumSMs) return 1;
+    if (rows <= 0 || rows >= 2 * kNumSMs) return 1;
     int64_t s = ceil_div(2 * kNumSMs, rows);
     s = std::min<int64_t>(s, ceil_div(items_per_row, 64));
     return int(std::max<int64_t>(1, std::min<int64_t>(s, 64)));
@@ -74,7 +74,7 @@ struct AttnPlan {
 // The tensor-core kernel runs one ~215 KB CTA per SM, so its splits fill the
 // 148 SMs in a single wave with at least one 64-item tile per split.
 static int choose_splits_tc(int64_t rows, int64_t items_per_row) {
-    if (rows >= kNumSMs) return 1;
+    if (rows <= 0 || rows >= kNumSMs) return 1;
     const int64_t s = std::min<int64_t>(kNumSMs / rows, ceil_div(items_per_row, 64));
     return int(std::max<int64_t>(1, std::min<int64_t>(s, 64)));
 }

@@ -103,3 +103,30 @@ def test_unbuilt_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(K, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         K.lib()
+
+
+def test_empty_inputs_are_no_ops_without_a_gpu():
+    """Zero tokens, rows or sequences: every entry point returns 0 before any
+    CUDA call (these run on CPU, where a CUDA call would fail)."""
+    lib = K.lib()
+    p = K.params(4, 128, 512, 64, 512, 64, 128, 0.044)
+    P = C.byref(p)
+    fake = C.c_void_p(0x1000)
+    assert lib.csa_compress(P, 64, fake, fake, fake, 0, K.F32, fake, None, None) == 0
+    assert lib.csa_quantize(K.FP8_S64, fake, 0, 64, fake, fake, None) == 0
+    assert lib.indexer_score(P, 0, 1, fake, fake, fake, fake, fake, 100, fake, fake, 100, None) == 0
+    assert lib.indexer_score(P, 1, 0, fake, fake, fake, fake, fake, 100, fake, fake, 100, None) == 0
+    assert lib.topk_select(P, 0, 1, fake, 10, 10, fake, fake, None) == 0
+    assert lib.topk_select(P, 1, 0, fake, 10, 10, fake, fake, None) == 0
+    assert lib.sparse_mqa_attn(P, 0, 1, fake, fake, fake, 10, fake, fake, 8, fake, fake, fake,
+                               fake, fake, 1 << 20, None) == 0
+    assert lib.hca_attn(P, 1, 0, fake, fake, fake, 10, fake, 8, fake, fake, fake,
+                        fake, fake, 1 << 20, None) == 0
+    assert lib.csa_decode(P, 0, fake, fake, fake, fake, fake, fake, fake, fake, 32768, fake, 128,
+                          fake, fake, fake, fake, fake, fake, 1 << 30, None) == 0
+    assert lib.csa_prefill(P, 1, 0, 0, fake, 64, 0, fake, fake, fake, fake, fake, fake, fake,
+                           fake, fake, fake, 100, fake, fake, fake, fake, 1 << 30, None) == 0
+    # workspace queries for empty batches plan no split (this once divided by zero)
+    for op in (K.OP_DECODE, K.OP_PREFILL, K.OP_SPARSE_ATTN, K.OP_HCA_ATTN):
+        assert 0 < lib.csa_workspace_size(P, op, 0, 1, 32768) < (1 << 20)
+        assert 0 < lib.csa_workspace_size(P, op, 3, 0, 32768) < (1 << 20)
