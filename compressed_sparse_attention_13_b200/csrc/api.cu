@@ -285,6 +285,15 @@ int hca_attn(const csa_params* p, int32_t batch, int32_t n_q, const void* q, con
 size_t csa_workspace_size(const csa_params* p, int32_t op, int32_t batch, int64_t n_q,
                           int64_t n_ctx) {
     if (!p || batch < 0 || n_q < 0 || n_ctx < 0 || p->n_heads <= 0 || p->head_dim <= 0) return 0;
+    // Every term below is at most rows x max(n_ctx, top_k + window, 64 x H x d) x 8 bytes
+    // (64 splits of fp32 partials); beyond size_t the answer saturates.
+    {
+        const unsigned __int128 rows_ = (unsigned __int128)batch * (uint64_t)n_q;
+        const int64_t per_row = std::max<int64_t>(std::max<int64_t>(n_ctx, int64_t(p->top_k) + p->window),
+                                                  int64_t(64) * p->n_heads * p->head_dim);
+        const unsigned __int128 per = (unsigned __int128)(uint64_t)per_row;
+        if (rows_ * per * 8 + (rows_ + 1) * 4096 > (unsigned __int128)(SIZE_MAX / 4)) return SIZE_MAX;
+    }
     const int64_t rows = int64_t(batch) * n_q;
     switch (op) {
     case CSA_OP_SPARSE_ATTN:

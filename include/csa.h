@@ -220,7 +220,8 @@ int csa_prefill(const csa_params* p, int32_t batch, int64_t T, int64_t t0, const
 #define CSA_OP_DECODE 2
 #define CSA_OP_PREFILL 3
 
-/* Bytes of workspace an operation needs (0 on bad arguments).  n_ctx is
+/* Bytes of workspace an operation needs (0 on bad arguments; SIZE_MAX when
+ * the size does not fit in size_t, which no buffer satisfies).  n_ctx is
  * max_entries (HCA) or max_blocks (decode, prefill); unused otherwise. */
 size_t csa_workspace_size(const csa_params* p, int32_t op, int32_t batch, int64_t n_q,
                           int64_t n_ctx);

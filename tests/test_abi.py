@@ -126,6 +126,11 @@ def test_empty_inputs_are_no_ops_without_a_gpu():
                           fake, fake, fake, fake, fake, fake, 1 << 30, None) == 0
     assert lib.csa_prefill(P, 1, 0, 0, fake, 64, 0, fake, fake, fake, fake, fake, fake, fake,
                            fake, fake, fake, 100, fake, fake, fake, fake, 1 << 30, None) == 0
+    # sizes beyond size_t saturate, so no buffer passes the workspace check
+    assert lib.csa_workspace_size(P, K.OP_PREFILL, 1 << 30, 1 << 40, 1 << 40) == 2 ** 64 - 1
+    assert lib.csa_prefill(P, 1 << 30, 1 << 30, 0, fake, 1 << 31, 0, fake, fake, fake, fake, fake,
+                           fake, fake, fake, fake, fake, 1 << 30, fake, fake, fake, fake,
+                           1 << 40, None) in (-1, -3, -4)
     # workspace queries for empty batches plan no split (this once divided by zero)
     for op in (K.OP_DECODE, K.OP_PREFILL, K.OP_SPARSE_ATTN, K.OP_HCA_ATTN):
         assert 0 < lib.csa_workspace_size(P, op, 0, 1, 32768) < (1 << 20)
