@@ -115,6 +115,8 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
     a.part_ml = (float2*)((char*)ws + plan.part_o_bytes);
     const bool tc = attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim) &&
                     attn_tc_rows_fit(max_entries, n_raw);
+    // the CUDA-core kernel puts the query rows on the grid's y axis
+    if (!tc && rows > kMaxGridY) return CSA_ERR_UNSUPPORTED;
     a.fused_combine = 0;
     a.row_base = 0;
     bool combined = false;
@@ -209,6 +211,8 @@ int indexer_score(const csa_params* p, int32_t batch, int32_t n_q, const void* q
     if (indexer_bf16_tc_supported(p->idx_fmt, p->idx_heads, p->idx_dim, max_blocks, batch, n_q))
         return cuda_status(launch_indexer_bf16_tc(qI, w, kI, max_blocks, q_pos, batch, n_q, p->m,
                                                   p->window, scores, ld_scores, (cudaStream_t)stream));
+    // the CUDA-core kernel puts the query rows on the grid's y axis
+    if (int64_t(batch) * n_q > kMaxGridY) return CSA_ERR_UNSUPPORTED;
     return cuda_status(launch_indexer_simt(p->idx_fmt, p->idx_heads, p->idx_dim, p->m, p->window,
                                            qI, qI_scales, w, kI, kI_scales, max_blocks, q_pos,
                                            batch, n_q, max_blocks, scores, ld_scores,

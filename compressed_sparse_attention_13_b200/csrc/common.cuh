@@ -15,6 +15,7 @@
 namespace csa {
 
 constexpr int kNumSMs = 148;  // B200
+constexpr int64_t kMaxGridY = 65535;  // largest grid extent along y (and z)
 
 // Device status word (CSA_DEV_* bits), shared by every call on a device.
 extern __device__ unsigned int g_status;

@@ -746,7 +746,7 @@ static cudaError_t launch_attn_tc_fmt(AttnArgs a, int64_t rows, cudaStream_t s, 
     cudaError_t e = ensure_smem(attn_tc_kernel<KVF>, sm);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.n_splits, unsigned(std::min<int64_t>(rows, 65535)));
+    cfg.gridDim = dim3(a.n_splits, unsigned(std::min<int64_t>(rows, kMaxGridY)));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = sm;
     cfg.stream = s;
@@ -773,11 +773,10 @@ static cudaError_t launch_attn_tc_fmt(AttnArgs a, int64_t rows, cudaStream_t s, 
     a.fused_combine = 0;
     cfg.attrs = pdl ? &attr[1] : nullptr;
     cfg.numAttrs = pdl ? 1 : 0;
-    // the grid's y extent is at most 65535: long prefill chunks take several launches
-    constexpr int64_t kMaxY = 65535;
-    for (int64_t r0 = 0; r0 < rows; r0 += kMaxY) {
+    // the grid's y extent is limited: long prefill chunks take several launches
+    for (int64_t r0 = 0; r0 < rows; r0 += kMaxGridY) {
         a.row_base = r0;
-        cfg.gridDim.y = unsigned(std::min(kMaxY, rows - r0));
+        cfg.gridDim.y = unsigned(std::min(kMaxGridY, rows - r0));
         e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<KVF>, map_q, map_win, map_kv, a);
         if (e != cudaSuccess) return e;
     }

@@ -123,6 +123,9 @@ int csa_quantize(int32_t fmt, const float* src, int64_t rows, int32_t d, void* o
  *   kI:        [batch][max_blocks][dI] in p->idx_fmt (+ kI_scales)
  *   q_pos:     int64 [batch][n_q]
  *   scores:    float [batch][n_q][ld_scores], ld_scores >= max_blocks
+ * Formats without a tensor-core path (F32, and BF16 with fewer than 4
+ * queries per sequence) take at most 65535 query rows (batch * n_q) per
+ * call; larger calls return CSA_ERR_UNSUPPORTED.
  * ------------------------------------------------------------------------ */
 int indexer_score(const csa_params* p, int32_t batch, int32_t n_q, const void* qI,
                   const void* qI_scales, const float* w, const void* kI, const void* kI_scales,
@@ -156,6 +159,10 @@ int topk_select(const csa_params* p, int32_t batch, int32_t n_q, const float* sc
  *   sinks:     float [H] or NULL
  *   out:       [batch][n_q][H][d] in p->act_fmt
  *   workspace: >= csa_workspace_size(p, CSA_OP_SPARSE_ATTN, batch, n_q, 0)
+ * The tensor-core path takes BF16 activations with FP8_S64 or BF16 entries
+ * at H = 64, d = 512; other shapes and formats take at most 65535 query
+ * rows (batch * n_q) per call (also for hca_attn, csa_decode and
+ * csa_prefill), larger calls returning CSA_ERR_UNSUPPORTED.
  * ------------------------------------------------------------------------ */
 int sparse_mqa_attn(const csa_params* p, int32_t batch, int32_t n_q, const void* q,
                     const void* kv, const void* kv_scales, int64_t max_entries,

@@ -135,3 +135,15 @@ def test_empty_inputs_are_no_ops_without_a_gpu():
     for op in (K.OP_DECODE, K.OP_PREFILL, K.OP_SPARSE_ATTN, K.OP_HCA_ATTN):
         assert 0 < lib.csa_workspace_size(P, op, 0, 1, 32768) < (1 << 20)
         assert 0 < lib.csa_workspace_size(P, op, 3, 0, 32768) < (1 << 20)
+
+
+def test_cuda_core_paths_refuse_more_rows_than_the_grid_holds():
+    """f32 attention and the CUDA-core indexer put query rows on the grid's y
+    axis (at most 65535): larger calls are refused on the host."""
+    lib = K.lib()
+    p = K.params(4, 64, 16, 8, 64, 4, 32, 0.125, act_fmt=K.F32, kv_fmt=K.F32, idx_fmt=K.F32)
+    P = C.byref(p)
+    fake = C.c_void_p(0x1000)
+    assert lib.sparse_mqa_attn(P, 2, 40000, fake, fake, None, 100, fake, fake, 8, fake, fake, None,
+                               fake, fake, 1 << 40, None) == -3
+    assert lib.indexer_score(P, 2, 40000, fake, None, fake, fake, None, 100, fake, fake, 100, None) == -3
