@@ -336,7 +336,6 @@ int csa_decode(const csa_params* p, int32_t batch, const void* q, const void* qI
     const size_t sel_bytes = ((size_t(batch) * p->top_k * 4) + 255) & ~size_t(255);
     void* ws_attn = (char*)workspace + sc_bytes + sel_bytes;
     const size_t ws_attn_bytes = ws_bytes - sc_bytes - sel_bytes;
-    cudaStream_t s = (cudaStream_t)stream;
     st = indexer_score(p, batch, 1, qI, qI_scales, w, kI, kI_scales, max_blocks, q_pos, scores, ld,
                        stream);
     if (st) return st;
@@ -347,7 +346,6 @@ int csa_decode(const csa_params* p, int32_t batch, const void* q, const void* qI
     if (st) return st;
     return sparse_attn_impl(p, batch, 1, q, kv, kv_scales, max_blocks, sel, raw, n_raw, raw_pos0,
                             q_pos, sinks, out, ws_attn, ws_attn_bytes, stream, false);
-    (void)s;
 }
 
 int csa_prefill(const csa_params* p, int32_t batch, int64_t T, int64_t t0, const void* raw,
