@@ -124,11 +124,14 @@ class Layer:
         t0 = self.t_next - T
         assert t0 % self.m == 0 and t0 == spec.prior_tokens, "one chunk, right after the prior cache"
         r0 = self._row(t0)
+        # only the chunk's complete blocks are pooled now; a partial last block
+        # is pooled by the decode step that completes it
+        nb = T // self.m
+        n_pool = nb * self.m
         if spec.kind == "csa":
             # indexer keys of the chunk's blocks first: csa_prefill reads them
-            nb = T // self.m
-            csa_compress(p, p.idx_dim, self.xI[r0:r0 + T], self.zI[r0:r0 + T], biasI, T,
-                         _rows(self.kI, t0 // self.m, nb))
+            csa_compress(p, p.idx_dim, self.xI[r0:r0 + n_pool], self.zI[r0:r0 + n_pool], biasI,
+                         n_pool, _rows(self.kI, t0 // self.m, nb))
             ws = torch.empty(csa_workspace_size(p, OP_PREFILL, 1, T, self.cap_blocks),
                              dtype=torch.uint8, device=q.device)
             rs = self._row(t0 - (self.W - 1)) if self.W > 0 else r0
@@ -136,8 +139,7 @@ class Layer:
                         bias, q, qI, w, self.kv, self.kI, self.cap_blocks, sinks, out, idx_out, ws)
             self._pooled = (t0 + T) // self.m
         else:
-            nb = T // self.m
-            csa_compress(p, self.d, self.x[r0:r0 + T], self.z[r0:r0 + T], bias, T,
+            csa_compress(p, self.d, self.x[r0:r0 + n_pool], self.z[r0:r0 + n_pool], bias, n_pool,
                          _rows(self.kv, t0 // self.m, nb))
             self._pooled = (t0 + T) // self.m
             q_pos = torch.arange(t0, t0 + T, dtype=torch.int64, device=q.device)
