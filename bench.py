@@ -50,17 +50,19 @@ def peaks():
 
 # ------------------------------------------------------------ algorithmic bytes
 def csa_decode_bytes(w):
-    """Bytes one CSA decode step must move (per batch): indexer keys of every
-    visible block (E2M1 + E8M0), the indexer query, the selected FP8 entries
-    (codes + scales), the bf16 window, q, and the bf16 output."""
+    """Bytes the method must move in one CSA decode step (per batch): the
+    indexer keys of every visible block (E2M1 + E8M0: 68 B at dI = 128), the
+    indexer query and weights, the selected FP8 entries (codes + scales), the
+    bf16 window, q, and the bf16 output.  The scores and the selection are
+    this design's intermediates, not the method's bytes, and are not counted."""
     nb = w.n_ctx // w.m
     ne = (w.n_ctx - w.W) // w.m
     key = w.dI // 2 + w.dI // 32
     ent = w.d + 4 * (w.d // 64)
-    per_seq = ne * key + w.HI * key + w.HI * 4 + w.k * ent + w.W * w.d * 2 + 2 * w.H * w.d * 2
-    return {"indexer": w.batch * (ne * key + w.HI * key + w.HI * 4 + ne * 4),
-            "attention": w.batch * (w.k * ent + w.W * w.d * 2 + 2 * w.H * w.d * 2),
-            "step": w.batch * per_seq, "n_blocks": nb}
+    idx = ne * key + w.HI * key + w.HI * 4
+    att = w.k * ent + w.W * w.d * 2 + 2 * w.H * w.d * 2
+    return {"indexer": w.batch * idx, "attention": w.batch * att, "step": w.batch * (idx + att),
+            "n_blocks": nb}
 
 
 def hca_decode_bytes(w):
@@ -79,10 +81,15 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, index: int, period: float = 0.002):
+    def __init__(self, index: int, period: float = 0.0005):
         self.index, self.period = index, period
         self.proc = self.thread = None
         self.samples, self.max_mhz, self.lines = [], None, []
+        self.marks = {}
+
+    def mark(self, name):
+        """Record the host time of an event (the timed region's start / end)."""
+        self.marks[name] = time.perf_counter()
 
     def _nvml_handle(self):
         import pynvml
@@ -111,7 +118,8 @@ class ClockSampler:
                     try:
                         sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
                         rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                        self.samples.append((sm, {n for n, b in bits.items() if rs & b}))
+                        self.samples.append((sm, {n for n, b in bits.items() if rs & b},
+                                             time.perf_counter()))
                     except Exception:
                         return
                     self.stop.wait(self.period)
@@ -150,14 +158,25 @@ class ClockSampler:
                     sm, self.max_mhz = float(f[1]), float(f[2])
                 except ValueError:
                     continue
-                self.samples.append((sm, {n for n, v in zip(self.NAMES, f[5:9]) if v.lower() == "active"}))
+                self.samples.append((sm, {n for n, v in zip(self.NAMES, f[5:9]) if v.lower() == "active"},
+                                     None))
 
     def summary(self):
-        sm = [x for x, _ in self.samples]
-        reasons = set().union(*(r for _, r in self.samples)) if self.samples else set()
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(reasons), "samples": len(sm),
-                "source": "nvml" if self.thread else ("nvidia-smi" if self.proc else None)}
+        """Median SM clock and the reasons seen over every sample (the whole
+        measurement: warm-up, timed steps and the per-kernel legs), plus the
+        same over the samples taken inside the timed region alone."""
+        sm = [x for x, _, _ in self.samples]
+        reasons = set().union(*(r for _, r, _ in self.samples)) if self.samples else set()
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+               "reasons": sorted(reasons), "samples": len(sm), "period_ms": self.period * 1e3,
+               "source": "nvml" if self.thread else ("nvidia-smi" if self.proc else None)}
+        t0, t1 = self.marks.get("timed_start"), self.marks.get("timed_end")
+        if t0 is not None and t1 is not None:
+            tr = [(x, r) for x, r, ts in self.samples if ts is not None and t0 <= ts <= t1]
+            out["timed_region"] = {"sm_mhz": statistics.median([x for x, _ in tr]) if tr else None,
+                                   "reasons": sorted(set().union(*(r for _, r in tr))) if tr else [],
+                                   "samples": len(tr), "seconds": round(t1 - t0, 4)}
+        return out
 
 
 # ------------------------------------------------------------------ our arm
@@ -219,8 +238,10 @@ def csa_decode_call(w, S, stream=None):
                  w.W, S["raw_pos0"], S["q_pos"], S["sinks"], S["out"], S["sel"], S["ws"], stream)
 
 
-def time_steps(fn, steps, warmup, flush, stream):
-    """Per-step CUDA-event times (ms) with an L2 flush before every step."""
+def time_steps(fn, steps, warmup, flush, stream, clk=None):
+    """Per-step CUDA-event times (ms) with an L2 flush before every step.
+    With a clock sampler, the timed region (after the warm-up, until the last
+    step has completed) is marked on it."""
     import torch
     for _ in range(warmup):
         flush.zero_()
@@ -228,13 +249,37 @@ def time_steps(fn, steps, warmup, flush, stream):
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
+    if clk is not None:
+        clk.mark("timed_start")
     for a, b in ev:
         flush.zero_()
         a.record(stream)
         fn()
         b.record(stream)
     torch.cuda.synchronize()
+    if clk is not None:
+        clk.mark("timed_end")
     return [a.elapsed_time(b) for a, b in ev]
+
+
+def kernel_times_in_step(fns, steps, warmup, flush, stream):
+    """Mean CUDA-event time (ms) of each of `fns`, run one after another as one
+    step (an L2 flush before every step), over `steps` steps after `warmup`."""
+    import torch
+    for _ in range(warmup):
+        flush.zero_()
+        for f in fns:
+            f()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)] for _ in range(steps)]
+    for e in ev:
+        flush.zero_()
+        e[0].record(stream)
+        for f, b in zip(fns, e[1:]):
+            f()
+            b.record(stream)
+    torch.cuda.synchronize()
+    return [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i in range(len(fns))]
 
 
 def graphed(fn):
@@ -296,7 +341,7 @@ def run_ours(args):
         flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
         legs = {"hca": lambda: bench_hca(args, dev, flush, stream, hbm_peak),
                 "prefill": lambda: bench_prefill(dev, flush, stream, bf16_peak),
-                "stack": lambda: bench_stack(dev, flush, stream, hbm_peak)}
+                "stack": lambda: bench_stack(dev, flush, stream, hbm_peak, bf16_peak)}
         print(json.dumps({n: legs[n]() for n in args.only_legs.split(",")}), flush=True)
         return
 
@@ -311,33 +356,60 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    # warm-up + timed steps (the clocks sampler runs across the timed region)
+    # warm-up + timed steps; the clock sampler runs across them and the
+    # per-kernel legs below, and marks the timed region
     barrier()
-    with ClockSampler(local) as clk:
-        times = time_steps(step, args.steps, args.warmup, flush, stream)
-        barrier()
+    clk = ClockSampler(local).__enter__()
+    times = time_steps(step, args.steps, args.warmup, flush, stream, clk)
+    barrier()
     t_ms = max_over_ranks(sum(times), dev)
     assert K.csa_device_status(reset=True) == 0
     value = job_throughput(w.batch, args.steps, world, t_ms)
 
-    # per-kernel times of the decode step (same launch configuration)
+    # The step's kernels one at a time: the three entry points csa_decode
+    # calls, with the same arguments (the same launches), enqueued eagerly with
+    # CUDA events between them on the launching stream, over the same number of
+    # steps, each step after an L2 flush.  The 256 MB flush runs for longer
+    # than the host takes to enqueue the step, so the events time the kernels,
+    # not the host.  Each is also timed alone (graph-replayed after a flush).
     nb = S["nb"]
     scores = S["ws"].view(torch.float32)[: w.batch * nb].view(w.batch, nb)
+    ws_attn = torch.empty(K.csa_workspace_size(S["p"], K.OP_SPARSE_ATTN, w.batch, 1, 0),
+                          dtype=torch.uint8, device=dev)
     kfn = {
         "indexer_score": lambda: K.indexer_score(S["p"], w.batch, 1, S["qI"], S["w"], S["kI"], nb,
                                                  S["q_pos"], scores, nb),
         "topk_select": lambda: K.topk_select(S["p"], w.batch, 1, scores, nb, nb, S["q_pos"], S["sel"]),
+        "sparse_mqa_attn": lambda: K.sparse_mqa_attn(
+            S["p"], w.batch, 1, S["q"], S["kv"], nb, S["sel"], S["window"], w.W, S["raw_pos0"],
+            S["q_pos"], S["sinks"], S["out"], ws_attn),
     }
-    ws_attn = torch.empty(K.csa_workspace_size(S["p"], K.OP_SPARSE_ATTN, w.batch, 1, 0),
-                          dtype=torch.uint8, device=dev)
-    kfn["sparse_mqa_attn"] = lambda: K.sparse_mqa_attn(
-        S["p"], w.batch, 1, S["q"], S["kv"], nb, S["sel"], S["window"], w.W, S["raw_pos0"],
-        S["q_pos"], S["sinks"], S["out"], ws_attn)
+    in_step = kernel_times_in_step(list(kfn.values()), args.steps, args.warmup, flush, stream)
+    in_step = dict(zip(kfn.keys(), in_step))
     kt = {name: statistics.mean(time_steps(graphed(fn), max(20, args.steps // 5), 3, flush, stream))
           for name, fn in kfn.items()}
+    clk.__exit__(None, None, None)
     by = csa_decode_bytes(w)
-    idx_gbs = by["indexer"] / (kt["indexer_score"] / 1e3) / 1e9
-    src = kernel_source_hash(["k_indexer_tc.cu", "sm100.cuh", "common.cuh"])
+    src = {"indexer_score": kernel_source_hash(["k_indexer_tc.cu", "sm100.cuh", "common.cuh"]),
+           "sparse_mqa_attn": kernel_source_hash(["k_attn_tc.cu", "sm100.cuh", "common.cuh"]),
+           "topk_select": kernel_source_hash(["k_topk.cu", "common.cuh"])}
+    kname = {"indexer_score": "indexer_tc_kernel", "sparse_mqa_attn": "attn_tc_kernel",
+             "topk_select": "topk"}
+    alg = {"indexer_score": by["indexer"], "sparse_mqa_attn": by["attention"]}
+    stage_roof = {}
+    for n, ms in in_step.items():
+        if n in alg:
+            gbs = alg[n] / (ms / 1e3) / 1e9
+            stage_roof[n] = {"kernel": kname[n], "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak,
+                             "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),
+                             "traffic": recorded_traffic(kname[n], src[n]), "algorithmic_bytes": alg[n],
+                             "us_in_step": round(ms * 1e3, 2), "peak_source": peak_kind}
+        else:
+            stage_roof[n] = {"kernel": kname[n], "bound": "latency", "us_in_step": round(ms * 1e3, 2),
+                             "score_bytes_read": w.batch * (by["n_blocks"] - w.W // w.m) * 4}
+    dominant = max(in_step, key=in_step.get)
+    if dominant not in alg:   # the roofline names an HBM-bound kernel; take the slower of the two
+        dominant = max(alg, key=lambda n: in_step[n])
 
     # end to end: host inputs (pinned) -> device, step, output -> host
     host = {n: S[n].detach().cpu().pin_memory() for n in ("q", "w", "window", "q_pos", "raw_pos0")}
@@ -368,11 +440,12 @@ def run_ours(args):
                    "head_dim": w.d, "idx_heads": w.HI, "idx_dim": w.dI, "m": w.m, "top_k": w.k,
                    "window": w.W, "kv": "fp8_e4m3_scale64", "indexer": "mxfp4",
                    "parallelism": f"replicas x{world}", "l2": "flushed (256 MB write) between steps"},
-        "roofline": {"kernel": "indexer_score (indexer_tc_kernel)", "bound": "hbm", "achieved": round(idx_gbs, 1),
-                     "peak": hbm_peak, "unit": "GB/s", "frac": round(idx_gbs / hbm_peak, 4),
-                     "traffic": recorded_traffic("indexer_tc_kernel", src),
-                     "algorithmic_bytes": by["indexer"], "peak_source": peak_kind},
-        "kernels_us": {n: round(v * 1e3, 2) for n, v in kt.items()},
+        # the slowest HBM-bound kernel of the step, timed inside the step
+        "roofline": dict(stage_roof[dominant], kernel=f"{dominant} ({kname[dominant]})"),
+        "stage_roofline": stage_roof,
+        "kernels_us_in_step": {n: round(v * 1e3, 2) for n, v in in_step.items()},
+        # each entry point alone, graph-replayed after an L2 flush (cold scores)
+        "kernels_us_isolated": {n: round(v * 1e3, 2) for n, v in kt.items()},
         "step_bytes": by["step"],
         "step_gbs": round(by["step"] / (t_ms / args.steps / 1e3) / 1e9, 1),
         "e2e": {"value": round(e2e_value, 1), "unit": "tok/s", "h2d_bytes_per_step": h2d,
@@ -388,7 +461,7 @@ def run_ours(args):
         del S
         torch.cuda.empty_cache()
         for key, name, leg in (("prefill_8k_bf16", "prefill", lambda: bench_prefill(dev, flush, stream, bf16_peak)),
-                               ("stack_c4", "stack", lambda: bench_stack(dev, flush, stream, hbm_peak))):
+                               ("stack_c4", "stack", lambda: bench_stack(dev, flush, stream, hbm_peak, bf16_peak))):
             if name not in legs:
                 continue
             try:
@@ -506,7 +579,7 @@ def bench_prefill(dev, flush, stream, bf16_peak):
                                "sparse_mqa_attn": roof("attn_tc_kernel<1> (bf16 entries)", tf_att)}}
 
 
-def bench_stack(dev, flush, stream, hbm_peak):
+def bench_stack(dev, flush, stream, hbm_peak, bf16_peak):
     """Four layers CSA, HCA, CSA, HCA on one sequence at 1M context: a prior
     cache of 1,044,480 tokens, a 4096-token prefill chunk, then 256 decode steps
     with incremental pooling (every 4 tokens for CSA, 128 for HCA)."""
@@ -599,19 +672,42 @@ def bench_stack(dev, flush, stream, hbm_peak):
     assert K.csa_device_status(reset=True) == 0
     del graph
     t_dec = statistics.median(dec) / STEPS
-    # algorithmic bytes of one decode step (four layers)
+    # algorithmic bytes of one decode step (four layers, at the middle step):
+    # CSA: 68 B per visible indexer key + the query and weights, the selected
+    # FP8 entries and the bf16 window; HCA: every visible FP8 entry + the window
     by = 0
     for ly in layers:
         t = PRIOR + CHUNK + STEPS // 2
         if ly["kind"] == "csa":
             ne = (t - W) // 4
-            by += ne * (64 + 4) + 2 * ne * 4 + TOPK * (d + 32) + W * d * 2 + 2 * H * d * 2
+            by += ne * (dI // 2 + dI // 32) + HI * (dI // 2 + dI // 32 + 4) + TOPK * (d + 4 * d // 64) + W * d * 2
         else:
             ne = (t - W) // 128
-            by += ne * (d + 32) + W * d * 2 + 2 * H * d * 2
+            by += ne * (d + 4 * d // 64) + W * d * 2
     gbs = by / (t_dec / 1e3) / 1e9
+    # work of the prefill chunk: the MXFP4 indexer (2 HI dI per visible
+    # (query, block) pair) and the bf16 attention (4 H d per attended item)
+    f_idx = f_att = 0
+    for ly in layers:
+        m = 4 if ly["kind"] == "csa" else 128
+        for t in range(PRIOR, PRIOR + CHUNK):
+            ne = max(0, (t - W) // m)
+            if ly["kind"] == "csa":
+                f_idx += ne * 2 * HI * dI
+                f_att += (min(TOPK, ne) + W) * 4 * H * d
+            else:
+                f_att += (ne + W) * 4 * H * d
+    fp4_peak = 4 * bf16_peak      # derived: the FP4 tensor rate is 4x the measured bf16 rate
+    roof_ms = (f_idx / fp4_peak + f_att / bf16_peak) / 1e12 * 1e3
     return {"workload": "csa_hca_stack_1m_4layers", "prior_tokens": PRIOR, "chunk": CHUNK, "decode_steps": STEPS,
             "prefill_ms": round(t_prefill, 3), "prefill_tok_s": round(CHUNK / (t_prefill / 1e3), 1),
+            "prefill_flop": {"indexer_mxfp4": f_idx, "attention_bf16": f_att},
+            "prefill_tflops": round((f_idx + f_att) / (t_prefill / 1e3) / 1e12, 1),
+            "prefill_roofline": {"bound": "tensor", "roofline_ms": round(roof_ms, 3),
+                                 "frac": round(roof_ms / t_prefill, 4),
+                                 "peaks_tflops": {"bf16": bf16_peak, "fp4": fp4_peak},
+                                 "note": "frac = time at the tensor peaks (indexer at the derived FP4 "
+                                         "peak, attention at the measured bf16 peak) / measured time"},
             "decode_us_per_step": round(t_dec * 1e3, 2), "decode_tok_s": round(1 / (t_dec / 1e3), 1),
             "decode_step_bytes": by,
             "roofline": {"kernel": "decode step (4 layers)", "bound": "hbm", "achieved": round(gbs, 1),
@@ -646,13 +742,22 @@ def _oracle_step(w, rows, sinks, threads):
         list(ex.map(one, rows))
 
 
+def host_threads() -> int:
+    """Host cores this process may run on (all of them for the CPU baseline)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
 def cpu_baseline(w, seconds):
-    """The oracle, as it stands, on all host cores: one sequence per thread,
+    """The oracle, as it stands (its source compiled -O3 -march=native with
+    OpenMP for this host), on all host cores: one sequence per thread,
     repeated until about `seconds` of CPU work."""
     import oracle
-    oracle.build()
-    cores = os.cpu_count() or 1
-    n = min(cores, 8)
+    oracle.use_native()
+    threads = host_threads()
+    n = min(threads, w.batch)
     rows, sinks = _oracle_sample(w, list(range(n)))
     t0 = time.perf_counter()
     reps = 0
@@ -662,8 +767,9 @@ def cpu_baseline(w, seconds):
         el = time.perf_counter() - t0
         if el * n >= seconds or el > seconds:
             break
-    return {"value": round(reps * n / el, 3), "unit": "tok/s", "cores": n, "kind": "oracle",
-            "sample": f"{reps} x {n} sequences of the {w.batch}-sequence batch (one thread each), "
+    return {"value": round(reps * n / el, 3), "unit": "tok/s", "cores": n, "host_cores": os.cpu_count(),
+            "threads": n, "kind": "oracle", "build": "g++ -O3 -march=native -fopenmp",
+            "sample": f"{reps} x {n} sequences of the {w.batch}-sequence batch (one per thread), "
                       f"{el:.1f} s wall"}
 
 
@@ -674,10 +780,10 @@ def run_reference(args):
         return
     import oracle
     from synth.workloads import WORKLOADS
-    oracle.build()
+    oracle.use_native()
     w = WORKLOADS[WORKLOAD]
-    cores = os.cpu_count() or 1
-    n = min(cores, 16)
+    threads = host_threads()
+    n = min(threads, w.batch)
     rows, sinks = _oracle_sample(w, list(range(n)))
     for _ in range(args.warmup):
         _oracle_step(w, rows, sinks, n)
@@ -693,8 +799,10 @@ def run_reference(args):
            "data": "synthetic (seeded N(0,1))",
            "config": {"workload": WORKLOAD, "batch": w.batch, "context": w.n_ctx, "heads": w.H,
                       "head_dim": w.d, "top_k": w.k, "window": w.W},
-           "cpu_baseline": {"value": round(value, 3), "unit": "tok/s", "cores": n, "kind": "oracle",
-                            "sample": f"each step: {n} of the {w.batch} sequences, one thread each"},
+           "cpu_baseline": {"value": round(value, 3), "unit": "tok/s", "cores": n,
+                            "host_cores": os.cpu_count(), "threads": n, "kind": "oracle",
+                            "build": "g++ -O3 -march=native -fopenmp",
+                            "sample": f"each step: {n} of the {w.batch} sequences, one per thread"},
            "e2e": {"value": round(value, 3), "unit": "tok/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)

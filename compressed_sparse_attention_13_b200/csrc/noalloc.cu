@@ -2,36 +2,28 @@
 // statically in this file, for callers that cannot allocate device memory.
 // Declared in include/csa.h, which lists the callers it serves and the
 // rules for using it.
-#include <mutex>
-
 #include "kernels.h"
 
 namespace {
 
 constexpr size_t kScratchBytes = CSA_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
-// One copy per device, reserved when the module loads; never freed.  Every
-// call writes each byte before reading it, so the contents at load do not
-// matter.
+// One copy per CUDA context that loads this library, reserved when the
+// module loads and freed only with the context.  Every call writes each byte
+// before reading it, so the contents at load do not matter.
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-std::mutex g_mu;
-void* g_scratch_of[kMaxDevices] = {};
-
-// Address of the scratch area on the current device, looked up once per
-// device with that device current.
-int scratch_on_current_device(void** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return CSA_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return CSA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_of[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return CSA_ERR_CUDA;
-        g_scratch_of[dev] = p;
-    }
-    *out = g_scratch_of[dev];
+// Device address of the scratch area in the context current on the calling
+// thread.  In host code the array's name is only a host-side stand-in, so the
+// address is asked of the runtime.  It is asked on every call instead of
+// being cached: a cached address would go stale after cudaDeviceReset (the
+// module reloads into a new context) or when the caller makes another context
+// current, and the lookup is a host-side table query once the module is
+// loaded (it may load the module on the first call in a context).
+int scratch_in_current_context(void** out) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return CSA_ERR_CUDA;
+    *out = p;
     return CSA_OK;
 }
 
@@ -50,7 +42,7 @@ extern "C" int csa_decode_noalloc(const csa_params* p, int32_t batch, const void
     if (csa_workspace_size(p, CSA_OP_DECODE, batch, 1, max_blocks) > kScratchBytes)
         return CSA_ERR_WORKSPACE;
     void* scratch = nullptr;
-    const int st = scratch_on_current_device(&scratch);
+    const int st = scratch_in_current_context(&scratch);
     if (st) return st;
     return csa_decode(p, batch, q, qI, qI_scales, w, kv, kv_scales, kI, kI_scales, max_blocks,
                       raw, n_raw, raw_pos0, q_pos, sinks, out, idx_out, scratch, kScratchBytes,

@@ -134,8 +134,10 @@ class Layer:
                          n_pool, _rows(self.kI, t0 // self.m, nb))
             ws = torch.empty(csa_workspace_size(p, OP_PREFILL, 1, T, self.cap_blocks),
                              dtype=torch.uint8, device=q.device)
-            rs = self._row(t0 - (self.W - 1)) if self.W > 0 else r0
-            csa_prefill(p, 1, T, t0, self.x[rs:], self.n_raw - rs, t0 - (self.W - 1), self.z[r0:r0 + T],
+            # first raw row the chunk's windows need (the chunk itself when W = 0)
+            rp0 = t0 - (self.W - 1) if self.W > 0 else t0
+            rs = self._row(rp0)
+            csa_prefill(p, 1, T, t0, self.x[rs:], self.n_raw - rs, rp0, self.z[r0:r0 + T],
                         bias, q, qI, w, self.kv, self.kI, self.cap_blocks, sinks, out, idx_out, ws)
             self._pooled = (t0 + T) // self.m
         else:

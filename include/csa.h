@@ -244,8 +244,8 @@ size_t csa_workspace_size(const csa_params* p, int32_t op, int32_t batch, int64_
  * It computes exactly what csa_decode computes, with the same kernels and
  * the same arguments, minus `workspace` and `ws_bytes`.  The scores,
  * selection and split-K partials go to a fixed scratch area that the library
- * reserves statically on each device: CSA_NOALLOC_SCRATCH_BYTES, which is
- * 32 MiB.  At m = 4, k = 512, W = 128 and 64 heads of 512, that covers any
+ * reserves statically in every CUDA context that loads it (one per device
+ * in the usual case): CSA_NOALLOC_SCRATCH_BYTES, which is 32 MiB.  At m = 4, k = 512, W = 128 and 64 heads of 512, that covers any
  * batch of 1 to 252 sequences of 128K tokens, or 32 sequences of up to
  * 500,000 tokens.  Nothing is allocated, not even on the first call.
  *
@@ -253,14 +253,16 @@ size_t csa_workspace_size(const csa_params* p, int32_t op, int32_t batch, int64_
  *           csa_workspace_size(p, CSA_OP_DECODE, batch, 1, max_blocks) is
  *           larger than CSA_NOALLOC_SCRATCH_BYTES.  Otherwise the errors are
  *           those of csa_decode.  CSA_ERR_CUDA if the scratch address cannot
- *           be found on the current device.
- *   device: the scratch belongs to the device that is current on the
- *           calling thread.  The stream and all pointers must belong to
- *           that device too.
- *   first call: on each device, the first call looks up the scratch's
- *           address.  That lookup may load the library's device code.  So
- *           make the first call on each device outside any stream capture,
- *           before the calls you intend to record.
+ *           be found in the current context.
+ *   device: the scratch belongs to the CUDA context that is current on
+ *           the calling thread (normally the device's primary context).  The
+ *           stream and all pointers must belong to that context too.  Its
+ *           address is looked up on every call, so a device reset or a
+ *           switch to another context is followed correctly.
+ *   first call: the first call in a context may load the library's device
+ *           code to find the scratch.  So make the first call on each device
+ *           outside any stream capture, before the calls you intend to
+ *           record.
  *   initial contents: none required.  Each scratch byte a call reads was
  *           written earlier in the same call, so nothing needs to start at
  *           zero.  The device status word (csa_device_status) is separate

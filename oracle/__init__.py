@@ -26,6 +26,9 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 
+_NATIVE = os.path.join(_HERE, "liboracle_native.so")
+
+
 def build(force: bool = False) -> str:
     """Compile the oracle (g++, -O2, OpenMP available but off unless asked)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
@@ -36,10 +39,32 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def build_native() -> str:
+    """Compile the same source for timing the CPU baseline on this host:
+    -O3 -march=native with OpenMP.  Always rebuilt, since the host's CPU decides
+    what -march=native means.  The arithmetic is the same source; only the
+    compiler's code generation differs."""
+    tmp = _NATIVE + f".tmp{os.getpid()}"
+    subprocess.check_call(["g++", "-O3", "-march=native", "-std=c++17", "-shared", "-fPIC",
+                           "-fopenmp", _SRC, "-o", tmp])
+    os.replace(tmp, _NATIVE)
+    return _NATIVE
+
+
+def use_native() -> None:
+    """Load the -O3 -march=native build in place of the parity build (for the
+    timed CPU baseline; the parity tests use the default build)."""
+    global _lib, _LIB
+    build_native()
+    _LIB, _lib = _NATIVE, None
+    lib()
+
+
 def lib():
     global _lib
     if _lib is None:
-        build()
+        if _LIB != _NATIVE:
+            build()
         L = C.CDLL(_LIB)
         P, I64, I32, D = C.c_void_p, C.c_int64, C.c_int, C.c_double
         L.orc_e4m3_value.restype = D

@@ -15,8 +15,9 @@ import torch
 import compressed_sparse_attention_13_b200 as K
 import oracle
 import synth
-from helpers import (FMT, act_dev, act_orc, assert_close_abs, assert_close_f32, both_stored,
-                     check_selection, down, orc_quantize, quant_codes_match, up)
+from helpers import (FMT, act_dev, act_orc, assert_attention_close, assert_close_abs, assert_close_f32,
+                     attention_bound_stored, bf16_values_match, both_stored, check_selection, down,
+                     orc_quantize, quant_codes_match, sink_dominant, up)
 
 pytestmark = pytest.mark.gpu
 
@@ -99,15 +100,9 @@ def test_compress_quantised_out(act, m, d, n_blocks, fmt):
     pre = oracle.compress(act_orc(x, act), act_orc(z, act), B, m)
     o = orc_quantize(pre, fmt)
     if fmt == "bf16":
-        # both sides round their own fp32 value to bf16; the fp32 values agree
-        # within 1e-5 of the row magnitude, so the stored values may differ by
-        # one bf16 ulp where a value sits on a rounding boundary, or by that
-        # absolute error for values that cancel to near zero
-        g = synth.bf16_bits_to_f32_np(down(st.data)).astype(np.float64)
-        r = synth.bf16_bits_to_f32_np(o.data).astype(np.float64)
-        row = np.max(np.abs(pre), axis=1, keepdims=True)
-        tol = np.maximum(2.0 ** -8 * np.abs(r), 1e-5 * row)
-        assert (np.abs(g - r) <= tol).all(), np.max(np.abs(g - r) - tol)
+        # both sides round their own fp32 value to bf16: values may differ
+        # only on a rounding boundary (within the fp32 rule of it)
+        assert bf16_values_match(down(st.data), o.data, pre) == 0
         return
     gs = down(st.scales)
     assert_close_f32(gs, o.scales, 1e-5, "scales")
@@ -247,12 +242,14 @@ def test_sparse_attention_matches_oracle(act, kvf, H, d, n_q, n_ent, W, k, m):
                       n_raw, up(raw_pos0), up(q_pos), up(sinks), out, ws)
     got = down(out.float())
     for b in range(batch):
-        ref = oracle.attention(act_orc(qv[b], act), orc_quantize(ent[b], kvf), idx[b],
-                               act_orc(raw[b], act), int(raw_pos0[b]), sinks, q_pos[b], H, m, W, scale)
+        args = (act_orc(qv[b], act), orc_quantize(ent[b], kvf), idx[b], act_orc(raw[b], act),
+                int(raw_pos0[b]))
+        ref = oracle.attention(*args, sinks, q_pos[b], H, m, W, scale)
         if act == "f32":
             assert_close_f32(got[b], ref, 1e-5, f"seq {b}")
         else:
-            assert_close_abs(got[b], ref, 2e-2, f"seq {b}")
+            bound = attention_bound_stored(*args, sinks, q_pos[b], H, m, W, scale)
+            assert_attention_close(got[b], ref, bound, f"seq {b}")
 
 
 @pytest.mark.parametrize("act,kvf,H,d,n_q,n_ent,W,m", [
@@ -274,12 +271,78 @@ def test_hca_attention_matches_oracle(act, kvf, H, d, n_q, n_ent, W, m):
                up(q_pos), up(sinks), out, ws)
     got = down(out.float())
     for b in range(batch):
-        ref = oracle.attention(act_orc(qv[b], act), orc_quantize(ent[b], kvf), None,
-                               act_orc(raw[b], act), int(raw_pos0[b]), sinks, q_pos[b], H, m, W, scale)
+        args = (act_orc(qv[b], act), orc_quantize(ent[b], kvf), None, act_orc(raw[b], act),
+                int(raw_pos0[b]))
+        ref = oracle.attention(*args, sinks, q_pos[b], H, m, W, scale)
         if act == "f32":
             assert_close_f32(got[b], ref, 1e-5, f"seq {b}")
         else:
-            assert_close_abs(got[b], ref, 2e-2, f"seq {b}")
+            bound = attention_bound_stored(*args, sinks, q_pos[b], H, m, W, scale)
+            assert_attention_close(got[b], ref, bound, f"seq {b}")
+
+
+# Rows whose outcome hinges on the sink and on each item: sink logits 2 above
+# every attended logit (the sink dominates the denominators), and positions
+# with few items: t < W (t + 1 raw tokens, no pooled entry) and t >= W with at
+# most three visible pooled blocks.  For each case the oracle also computes the
+# two mistakes these rows are there to catch -- the sink left out, and the
+# window one token short (or the query's own token left out) -- and the test
+# first checks that each of those misses the tolerance, so that a kernel
+# making it would fail.
+@pytest.mark.parametrize("kvf,dense,n_splits_hint", [
+    ("fp8", False, "few rows: splits combined in the cluster"),
+    ("bf16", False, "bf16 entries gathered by the converters"),
+    ("fp8", True, "HCA: dense entries"),
+])
+def test_attention_sink_dominant_and_few_item_rows(kvf, dense, n_splits_hint):
+    H, d, m, W, k, seed = 64, 512, 4, 128, 16, 31
+    scale = 1 / math.sqrt(d)
+    n_ent, batch = 3, 2
+    # sequence 0: positions below the window; sequence 1: t >= W with <= 3 blocks
+    q_pos = np.array([[0, 1, 5, 17, 40, 126], [W, W + 1, W + m, W + 2 * m + 1, W + 3 * m, W + 3 * m + 3]],
+                     np.int64)
+    n_q = q_pos.shape[1]
+    n_raw = W + 3 * m + 4
+    raw_pos0 = np.zeros(batch, np.int64)
+    qv = synth.tensor_np(seed, "sq", (batch, n_q, H, d), dtype="bf16")
+    ent = synth.tensor_np(seed, "skv", (batch, n_ent, d))
+    raw = synth.tensor_np(seed, "sraw", (batch, n_raw, d), dtype="bf16")
+    idx = np.full((batch, n_q, k), -1, np.int32)
+    for b in range(batch):
+        for i in range(n_q):
+            ne = min(oracle.n_elig(int(q_pos[b, i]), m, W), n_ent)
+            idx[b, i, :ne] = np.arange(ne)
+    kd, _ = both_stored(ent.reshape(-1, d), kvf)
+    orc_in = [(act_orc(qv[b], "bf16"), orc_quantize(ent[b], kvf), None if dense else idx[b],
+               act_orc(raw[b], "bf16"), 0) for b in range(batch)]
+    sinks = np.max([sink_dominant(*orc_in[b], q_pos[b], H, m, W, scale) for b in range(batch)], axis=0)
+    p = K.params(m, W, k, H, d, 1, 32, scale, act_fmt=K.BF16, kv_fmt=FMT[kvf])
+    out = torch.empty((batch, n_q, H, d), dtype=torch.bfloat16, device="cuda")
+    args = (p, batch, n_q, act_dev(qv, "bf16"), kd, n_ent)
+    tail = (act_dev(raw, "bf16"), n_raw, up(raw_pos0), up(q_pos), up(sinks), out)
+    if dense:
+        ws = torch.empty(K.csa_workspace_size(p, K.OP_HCA_ATTN, batch, n_q, n_ent), dtype=torch.uint8,
+                         device="cuda")
+        K.hca_attn(*args, *tail, ws)
+    else:
+        ws = torch.empty(K.csa_workspace_size(p, K.OP_SPARSE_ATTN, batch, n_q, 0), dtype=torch.uint8,
+                         device="cuda")
+        K.sparse_mqa_attn(*args, up(idx), *tail, ws)
+    got = down(out.float())
+    for b in range(batch):
+        ref = oracle.attention(*orc_in[b], sinks, q_pos[b], H, m, W, scale)
+        bound = attention_bound_stored(*orc_in[b], sinks, q_pos[b], H, m, W, scale)
+        # the planted mistakes (on the CPU) miss the tolerance on every row
+        no_sink = oracle.attention(*orc_in[b], np.full(H, -np.inf, np.float32), q_pos[b], H, m, W, scale)
+        assert ((np.abs(no_sink - ref) > bound).any(axis=(1, 2))).all()
+        if b == 0:
+            short = oracle.attention(*orc_in[b], sinks, q_pos[b] - 1, H, m, W, scale)  # own token left out
+            rows = q_pos[b] >= 1
+        else:
+            short = oracle.attention(*orc_in[b], sinks, q_pos[b], H, m, W - 1, scale)
+            rows = np.ones(n_q, bool)
+        assert ((np.abs(short - ref) > bound).any(axis=(1, 2)))[rows].all()
+        assert_attention_close(got[b], ref, bound, f"seq {b}")
 
 
 def test_out_of_range_index_is_flagged_not_read():

@@ -10,11 +10,18 @@ import torch
 import compressed_sparse_attention_13_b200 as K
 import oracle
 import synth
-from helpers import (FMT, act_dev, act_orc, assert_close_abs, assert_close_f32, both_stored,
-                     check_selection, down, orc_quantize, up)
+from helpers import (FMT, act_dev, act_orc, assert_attention_close, assert_close_abs, assert_close_f32,
+                     attention_bound_stored, both_stored, check_selection, down, orc_quantize,
+                     sink_dominant, up)
 from synth.workloads import WORKLOADS, draw_np
 
 pytestmark = pytest.mark.gpu
+
+
+def _threads():
+    """Oracle threads for the larger checks (independent query rows)."""
+    import os
+    return max(1, len(os.sched_getaffinity(0)))
 
 
 @pytest.fixture(autouse=True)
@@ -24,7 +31,7 @@ def _clean_status():
     assert K.csa_device_status(reset=True) == 0
 
 
-def run_decode_case(w, q_pos, check_rows=None):
+def run_decode_case(w, q_pos, check_rows=None, sink_shift=None):
     """CSA decode through csa_decode; returns (out, sel) on the host plus the
     oracle-side stored inputs for checking."""
     B, H, d, HI, dI, m, W, k = w.batch, w.H, w.d, w.HI, w.dI, w.m, w.W, w.k
@@ -42,6 +49,11 @@ def run_decode_case(w, q_pos, check_rows=None):
     qI_d, _ = both_stored(qI.reshape(-1, dI), w.idx)
     q_pos = np.asarray(q_pos, np.int64)
     raw_pos0 = q_pos - W + 1
+    if sink_shift is not None:
+        # sinks above every logit any selection could contain (all visible blocks)
+        sinks = np.max([sink_dominant(act_orc(q[b], w.act), orc_quantize(kv[b], w.kv), None,
+                                      act_orc(win[b], w.act), int(raw_pos0[b]), [int(q_pos[b])],
+                                      H, m, W, w.scale, sink_shift) for b in range(B)], axis=0)
     out = torch.empty((B, H, d), dtype=torch.bfloat16 if w.act == "bf16" else torch.float32,
                       device="cuda")
     sel = torch.empty((B, k), dtype=torch.int32, device="cuda")
@@ -59,12 +71,13 @@ def run_decode_case(w, q_pos, check_rows=None):
         ne = min(oracle.n_elig(t, m, W), nb)
         check_selection(got_sel[b], scores, ne, k, what=f"seq {b}")
         # output against the oracle's attention over the library's (valid) selection
-        ref = oracle.attention(act_orc(q[b], w.act), kv_o, got_sel[b][None], act_orc(win[b], w.act),
-                               t - W + 1, sinks, [t], H, m, W, w.scale)[0]
+        args = (act_orc(q[b], w.act), kv_o, got_sel[b][None], act_orc(win[b], w.act), t - W + 1)
+        ref = oracle.attention(*args, sinks, [t], H, m, W, w.scale)[0]
         if w.act == "f32":
             assert_close_f32(got[b], ref, 1e-5, f"seq {b}")
         else:
-            assert_close_abs(got[b], ref, 2e-2, f"seq {b}")
+            bound = attention_bound_stored(*args, sinks, [t], H, m, W, w.scale)[0]
+            assert_attention_close(got[b], ref, bound, f"seq {b}")
     return got, got_sel
 
 
@@ -73,6 +86,13 @@ def test_csa_decode_reduced_ragged():
     # ragged: full context, partial, fewer eligible blocks than k, none eligible
     q_pos = [8192, 8000, 4 * 300 + 128, 50]
     run_decode_case(w, q_pos)
+
+
+def test_csa_decode_sink_dominant():
+    """Sink logits 2 above every attended logit: the outputs shrink by about
+    e^-2 and a mishandled sink fails both matching rules."""
+    w = WORKLOADS["csa_decode_128k_b32"].with_(batch=3, n_ctx=4096, seed=14)
+    run_decode_case(w, [4096, 2500, 4 * 200 + 128], sink_shift=2.0)
 
 
 def test_csa_decode_degenerate_all_blocks_no_window():
@@ -135,12 +155,13 @@ def _run_prefill(w, check_every):
             ne = min(oracle.n_elig(int(t), m, W), nb)
             check_selection(got_sel[b, t], scores[a], ne, k, what=f"seq {b} t {t}")
         q_rows = q[b][rows]
-        ref = oracle.attention(act_orc(q_rows.reshape(-1, d), w.act), kv_o, got_sel[b][rows],
-                               act_orc(x[b], w.act), 0, sinks, rows, H, m, W, w.scale)
+        args = (act_orc(q_rows.reshape(-1, d), w.act), kv_o, got_sel[b][rows], act_orc(x[b], w.act), 0)
+        ref = oracle.attention(*args, sinks, rows, H, m, W, w.scale, n_threads=_threads())
         if w.act == "f32":
             assert_close_f32(got[b][rows], ref, 1e-5, f"prefill seq {b}")
         else:
-            assert_close_abs(got[b][rows], ref, 2e-2, f"prefill seq {b}")
+            bound = attention_bound_stored(*args, sinks, rows, H, m, W, w.scale)
+            assert_attention_close(got[b][rows], ref, bound, f"prefill seq {b}")
 
 
 def test_hca_decode_reduced():
@@ -177,7 +198,8 @@ def _run_hca(w, check_batches, draw_on_device=False):
         pooled = oracle.compress(act_orc(xb, w.act), act_orc(zb, w.act), bias, m)
         kv_o = orc_quantize(pooled, w.kv)
         win = np.concatenate([xb[N - W + 1:], x_new[b][None]])
-        ref = oracle.attention(act_orc(q[b], w.act), kv_o, None, act_orc(win, w.act), N - W + 1,
-                               sinks, [N], H, m, W, w.scale)[0]
-        assert_close_abs(got[b], ref, 2e-2, f"hca seq {b}")
+        args = (act_orc(q[b], w.act), kv_o, None, act_orc(win, w.act), N - W + 1)
+        ref = oracle.attention(*args, sinks, [N], H, m, W, w.scale)[0]
+        bound = attention_bound_stored(*args, sinks, [N], H, m, W, w.scale)[0]
+        assert_attention_close(got[b], ref, bound, f"hca seq {b}")
     return got

@@ -1,7 +1,8 @@
 """csa_decode_noalloc: the same decode step as csa_decode, computed on the
 library's fixed device scratch instead of a caller workspace.  Two calls in a
-row on different inputs must each agree with csa_decode on the same inputs,
-and a request larger than the scratch is refused on the host."""
+row on different inputs must each give exactly what csa_decode gives on the
+same inputs (same kernels, same arithmetic: bitwise equal), and a request
+larger than the scratch is refused on the host."""
 import ctypes as C
 
 import numpy as np
@@ -9,7 +10,7 @@ import pytest
 import torch
 
 import compressed_sparse_attention_13_b200 as K
-from helpers import FMT, act_dev, assert_close_abs, both_stored, down, up
+from helpers import FMT, act_dev, both_stored, down, up
 from synth.workloads import WORKLOADS, draw_np
 
 
@@ -62,7 +63,7 @@ def test_noalloc_matches_csa_decode_on_two_calls_in_a_row():
                              w.W, a["raw_pos0"], a["q_pos"], a["sinks"], out, sel)
         got_sel, want_sel = down(sel), down(ref_sel)
         assert np.array_equal(got_sel, want_sel), f"seed {seed}: selections differ"
-        got, want = down(out.float()), down(ref_out.float())
-        for b in range(w.batch):
-            assert_close_abs(got[b], want[b], 2e-2, f"seed {seed} seq {b}")
+        # the same kernels on the same inputs: the outputs are bitwise equal
+        got, want = down(out), down(ref_out)
+        assert np.array_equal(got, want), f"seed {seed}: outputs differ"
         assert K.csa_device_status(reset=True) == 0
