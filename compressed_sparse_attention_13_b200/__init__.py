@@ -7,7 +7,7 @@ Importing works without a GPU (the library loads, nothing launches); calling
 anything without the built library raises.
 
 Names follow the C ABI: ``csa_compress``, ``csa_quantize``, ``indexer_score``,
-``topk_select``, ``sparse_mqa_attn``, ``hca_attn``, ``csa_decode``,
+``topk_select``, ``sparse_mqa_attn``, ``hca_attn``, ``window_attn``, ``csa_decode``,
 ``csa_prefill``, ``csa_workspace_size``, ``csa_device_status``, and
 ``csa_decode_noalloc`` (csa_decode on the library's fixed device scratch, for
 callers that cannot allocate).
@@ -19,7 +19,8 @@ import os
 from dataclasses import dataclass
 
 F32, BF16, FP8_S64, MXFP4 = 0, 1, 2, 3
-OP_SPARSE_ATTN, OP_HCA_ATTN, OP_DECODE, OP_PREFILL = 0, 1, 2, 3
+OP_SPARSE_ATTN, OP_HCA_ATTN, OP_DECODE, OP_PREFILL, OP_WINDOW_ATTN = 0, 1, 2, 3, 4
+FLAG_BATCH_INVARIANT = 0x1
 DEV_BAD_INDEX, DEV_RANGE, DEV_TIMEOUT = 0x1, 0x2, 0x4
 NOALLOC_SCRATCH_BYTES = 32 << 20   # CSA_NOALLOC_SCRATCH_BYTES
 ERR_WORKSPACE = -4
@@ -40,18 +41,18 @@ class Params(C.Structure):
     _fields_ = [("m", C.c_int32), ("window", C.c_int32), ("top_k", C.c_int32),
                 ("n_heads", C.c_int32), ("head_dim", C.c_int32), ("idx_heads", C.c_int32),
                 ("idx_dim", C.c_int32), ("scale", C.c_float), ("act_fmt", C.c_int32),
-                ("kv_fmt", C.c_int32), ("idx_fmt", C.c_int32)]
+                ("kv_fmt", C.c_int32), ("idx_fmt", C.c_int32), ("flags", C.c_uint32)]
 
 
 def params(m, window, top_k, n_heads, head_dim, idx_heads, idx_dim, scale,
-           act_fmt=BF16, kv_fmt=FP8_S64, idx_fmt=MXFP4) -> Params:
+           act_fmt=BF16, kv_fmt=FP8_S64, idx_fmt=MXFP4, flags=0) -> Params:
     return Params(m, window, top_k, n_heads, head_dim, idx_heads, idx_dim, float(scale),
-                  act_fmt, kv_fmt, idx_fmt)
+                  act_fmt, kv_fmt, idx_fmt, flags)
 
 
 EXPORTS = ["csa_compress", "csa_quantize", "indexer_score", "topk_select", "sparse_mqa_attn",
-           "hca_attn", "csa_decode", "csa_prefill", "csa_workspace_size", "csa_device_status",
-           "csa_strerror", "csa_version", "csa_decode_noalloc"]
+           "hca_attn", "window_attn", "csa_decode", "csa_prefill", "csa_workspace_size",
+           "csa_device_status", "csa_strerror", "csa_version", "csa_decode_noalloc"]
 
 
 def lib():
@@ -70,6 +71,7 @@ def lib():
         L.sparse_mqa_attn.argtypes = [PP, I32, I32, P, P, P, I64, P, P, I64, P, P, P, P, P,
                                       C.c_size_t, P]
         L.hca_attn.argtypes = [PP, I32, I32, P, P, P, I64, P, I64, P, P, P, P, P, C.c_size_t, P]
+        L.window_attn.argtypes = [PP, I32, I32, P, P, I64, P, P, P, P, P, C.c_size_t, P]
         L.csa_decode.argtypes = [PP, I32, P, P, P, P, P, P, P, P, I64, P, I64, P, P, P, P, P, P,
                                  C.c_size_t, P]
         L.csa_prefill.argtypes = [PP, I32, I64, I64, P, I64, I64, P, P, P, P, P, P, P, P, P, P,
@@ -186,6 +188,14 @@ def hca_attn(p: Params, batch: int, n_q: int, q, kv: Stored, max_entries: int, r
     _ok("hca_attn", lib().hca_attn(
         C.byref(p), batch, n_q, _p(q), _p(kv.data), _p(kv.scales), max_entries, _p(raw), n_raw,
         _p(raw_pos0), _p(q_pos), _p(sinks), _p(out), wp, wb, _s(stream)))
+
+
+def window_attn(p: Params, batch: int, n_q: int, q, raw, n_raw: int, raw_pos0, q_pos, sinks, out,
+                workspace=None, stream=None):
+    wp, wb = _ws(workspace)
+    _ok("window_attn", lib().window_attn(
+        C.byref(p), batch, n_q, _p(q), _p(raw), n_raw, _p(raw_pos0), _p(q_pos), _p(sinks), _p(out),
+        wp, wb, _s(stream)))
 
 
 def csa_decode(p: Params, batch: int, q, qI: Stored, w, kv: Stored, kI: Stored, max_blocks: int,

@@ -38,6 +38,7 @@ static bool idx_ok(int f) { return f == CSA_F32 || f == CSA_BF16 || f == CSA_MXF
 static int check_params(const csa_params* p, bool need_idx, bool need_attn) {
     if (!p) return CSA_ERR_ARG;
     if (p->m <= 0 || p->window < 0) return CSA_ERR_ARG;
+    if (p->flags & ~CSA_FLAG_BATCH_INVARIANT) return CSA_ERR_ARG;
     if (need_attn) {
         if (p->n_heads <= 0 || p->head_dim <= 0 || (p->head_dim % 64) != 0) return CSA_ERR_ARG;
         if (!act_ok(p->act_fmt) || !kv_ok(p->kv_fmt)) return CSA_ERR_ARG;
@@ -79,13 +80,25 @@ static int choose_splits_tc(int64_t rows, int64_t items_per_row) {
     return int(std::max<int64_t>(1, std::min<int64_t>(s, 64)));
 }
 
+// Batch-invariant mode: the split count of a row depends on the row's own
+// number of items only (never on how many rows share the launch), so a row's
+// partial sums, their combine order and hence its output bits are the same
+// in any batch.  About three 64-item tiles per split, at most 8 (one cluster).
+static int choose_splits_invariant(int64_t items_per_row) {
+    const int64_t tiles = ceil_div(std::max<int64_t>(items_per_row, 1), 64);
+    return int(std::max<int64_t>(1, std::min<int64_t>(8, ceil_div(tiles, 3))));
+}
+
 static AttnPlan plan_attn(const csa_params* p, int64_t rows, int64_t items_per_row) {
     AttnPlan a;
     // (the tensor-core kernel is also limited to rows that fit 32 bits; with
     // larger buffers the CUDA-core kernel runs with the same split count)
-    a.n_splits = attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim)
-                     ? choose_splits_tc(rows, items_per_row)
-                     : choose_splits(rows, items_per_row);
+    if (p->flags & CSA_FLAG_BATCH_INVARIANT)
+        a.n_splits = choose_splits_invariant(items_per_row);
+    else
+        a.n_splits = attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim)
+                         ? choose_splits_tc(rows, items_per_row)
+                         : choose_splits(rows, items_per_row);
     const int64_t items = rows * a.n_splits;
     a.part_o_bytes = size_t(items) * p->n_heads * p->head_dim * sizeof(float);
     a.part_ml_bytes = size_t(items) * p->n_heads * sizeof(float2);
@@ -146,10 +159,10 @@ static cudaError_t launch_fill_positions(int64_t* q_pos, int64_t* pos0, int batc
 
 static int check_attn_ptrs(const void* q, const void* kv, const void* kv_s, int kv_fmt,
                            const void* raw, int64_t n_raw, const int64_t* raw_pos0,
-                           const int64_t* q_pos, void* out) {
-    if (!q || !kv || !q_pos || !out || !raw_pos0) return CSA_ERR_ARG;
+                           const int64_t* q_pos, void* out, bool need_kv = true) {
+    if (!q || (need_kv && !kv) || !q_pos || !out || !raw_pos0) return CSA_ERR_ARG;
     if (n_raw < 0 || (n_raw > 0 && !raw)) return CSA_ERR_ARG;
-    if (kv_fmt == CSA_FP8_S64 && !kv_s) return CSA_ERR_ARG;
+    if (need_kv && kv_fmt == CSA_FP8_S64 && !kv_s) return CSA_ERR_ARG;
     if (!aligned16(q) || !aligned16(kv) || !aligned16(kv_s) || !aligned16(raw) || !aligned16(out))
         return CSA_ERR_ALIGN;
     return CSA_OK;
@@ -286,6 +299,21 @@ int hca_attn(const csa_params* p, int32_t batch, int32_t n_q, const void* q, con
                     (cudaStream_t)stream);
 }
 
+int window_attn(const csa_params* p, int32_t batch, int32_t n_q, const void* q, const void* raw,
+                int64_t n_raw, const int64_t* raw_pos0, const int64_t* q_pos, const float* sinks,
+                void* out, void* workspace, size_t ws_bytes, csa_stream_t stream) {
+    int st = check_params(p, false, true);
+    if (st) return st;
+    if (batch < 0 || n_q < 0) return CSA_ERR_ARG;
+    if (batch == 0 || n_q == 0) return CSA_OK;
+    st = check_attn_ptrs(q, nullptr, nullptr, p->kv_fmt, raw, n_raw, raw_pos0, q_pos, out, false);
+    if (st) return st;
+    // no pooled entry is visible: the dense path over zero entries attends the
+    // window (and the sink) alone
+    return run_attn(p, batch, n_q, q, nullptr, nullptr, 0, nullptr, raw, n_raw, raw_pos0, q_pos, sinks,
+                    out, workspace, ws_bytes, p->window, (cudaStream_t)stream);
+}
+
 size_t csa_workspace_size(const csa_params* p, int32_t op, int32_t batch, int64_t n_q,
                           int64_t n_ctx) {
     if (!p || batch < 0 || n_q < 0 || n_ctx < 0 || p->n_heads <= 0 || p->head_dim <= 0) return 0;
@@ -304,6 +332,8 @@ size_t csa_workspace_size(const csa_params* p, int32_t op, int32_t batch, int64_
         return plan_attn(p, rows, int64_t(p->top_k) + p->window).bytes() + 256;
     case CSA_OP_HCA_ATTN:
         return plan_attn(p, rows, n_ctx + p->window).bytes() + 256;
+    case CSA_OP_WINDOW_ATTN:
+        return plan_attn(p, rows, p->window).bytes() + 256;
     case CSA_OP_DECODE:
     case CSA_OP_PREFILL: {
         const size_t pos = op == CSA_OP_PREFILL ? ((size_t(rows) + batch) * 8 + 255) & ~size_t(255) : 0;

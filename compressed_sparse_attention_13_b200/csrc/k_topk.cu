@@ -1,13 +1,14 @@
 // Top-k block selection ("DeepSeek V4" wiki summary, section 架构创新: the
 // lightning indexer makes a top-k sparse selection of pooled entries).
 //
-// Radix select on the order-preserving 32-bit image of each fp32 score: three
-// histogram passes over 11, 11 and 10 bits find the exact k-th largest key
-// T and how many elements equal to T are needed; a final pass writes every
-// element above T and the first needed elements equal to T, in ascending
-// index order, so ties resolve to the lower index.  -0.0 is folded into +0.0
-// before ranking.  One 1024-thread CTA per query row; rows are read from
-// global memory (an L2-resident score row in the decode path).
+// Every kernel here ranks the order-preserving 32-bit image of each fp32 score
+// (-0.0 folded into +0.0), finds the exact k-th largest key T by radix passes
+// and how many keys equal to T are taken, and writes the selected ids in
+// ascending order, ties going to the lower index.  Rows of up to 32,768
+// scores (decode at 128K context, prefill chunks) take topk_sel_kernel, which
+// narrows the row to a few times k candidates with a sampled threshold
+// first; longer rows take a thread-block cluster per row (few rows) or one
+// CTA per row reading the row from global memory (many rows).
 #include <cooperative_groups.h>
 
 #include "kernels.h"
@@ -390,6 +391,478 @@ __global__ void __cluster_dims__(kClu, 1, 1) __launch_bounds__(kCluThreads)
     cluster.sync();  // keep this CTA's shared memory alive until every remote read is done
 }
 
+// Rows of any length with a sampled threshold (topk_sel_kernel): a cluster of
+// CPR CTAs per row (one CTA for short rows), CTA r holding keys [r SEG,
+// (r+1) SEG) of the row, SEG = 4 V kSelThreads, loaded as float4 chunks (chunk
+// u of thread t: keys 4 (u kSelThreads + t) .. + 3 of the segment).
+//  1. each CTA builds an 11-bit histogram of a sample of its keys (chunk 0 of
+//     every thread) and takes a threshold bin b_r such that, by a wide margin,
+//     its segment's share of the row's top k lies in bins >= b_r (rows of at
+//     most 4096 keys take every key: b_r = 0);
+//  2. each CTA pushes its keys in bins >= b_r, as (key, id) pairs, into the
+//     candidate area of the cluster's first CTA (the leader), one remote
+//     slot reservation per warp, and records b_r there;
+//  3. the leader finds the exact k-th largest candidate T (four 8-bit radix
+//     passes, lanes with equal digits merged before the shared atomics) and
+//     how many candidates equal to T are taken; if more equal T than are
+//     taken, a radix select over their complemented ids keeps the lowest ids;
+//  4. the selected ids are marked in a bitmap of the row and written in
+//     ascending order (a block scan of the bitmap words' population counts).
+// The selection is exact when T >= every CTA's threshold (any key left out
+// then lies below T) and the candidates fit; otherwise the leader runs an
+// exact radix select over the whole row in global memory instead.
+constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelCap = 8192;           // most candidates kept in the leader's shared memory
+constexpr int kSelNoSampleMax = 4096;   // rows this short take every key as a candidate
+
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Histogram add from a whole warp: lanes holding the same bin are merged so
+// that one leader adds their count (candidates share most of their top bits).
+__device__ __forceinline__ void warp_hist_add(int* hist, bool in, uint32_t bin) {
+    const uint32_t dg = in ? bin : 0xFFFFFFFFu;
+    const unsigned same = __match_any_sync(0xffffffffu, dg);
+    if (in && (threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[dg], __popc(same));
+}
+
+// The k-th largest value among v[0..C) passing `keep` (1 <= k <= their
+// number): four 8-bit radix passes over the whole CTA.  Returns the value T,
+// how many values equal to T are among the k largest (rem) and how many
+// equal T (eq).
+template <typename Keep>
+__device__ __forceinline__ void sel_radix(const uint32_t* v, int C, int k, Keep keep, int* hist,
+                                          int* sh, uint32_t& T, int& rem, int& eq) {
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = k;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        if (tid < 256) hist[tid] = 0;
+        __syncthreads();
+        for (int i0 = 0; i0 < C; i0 += kSelThreads) {  // whole warps iterate together
+            const int i = i0 + tid;
+            const uint32_t u = i < C ? v[i] : 0u;
+            warp_hist_add(hist, i < C && (u & pmask) == prefix && keep(i), (u >> shift) & 255u);
+        }
+        __syncthreads();
+        if (wid == 0) {
+            // lane l owns the 8 bins 255-8l .. 248-8l (counted from the top)
+            int loc[8], sum = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { loc[j] = hist[255 - 8 * lane - j]; sum += loc[j]; }
+            int inc = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int x = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += x;
+            }
+            int above = inc - sum;
+            if (above < remaining && remaining <= inc) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (above < remaining && remaining <= above + loc[j]) {
+                        sh[0] = 255 - 8 * lane - j;
+                        sh[1] = above;
+                        sh[2] = loc[j];
+                    }
+                    above += loc[j];
+                }
+            }
+        }
+        __syncthreads();
+        remaining -= sh[1];
+        prefix |= uint32_t(sh[0]) << shift;
+        pmask |= 0xFFu << shift;
+        eq = sh[2];
+        __syncthreads();  // sh is rewritten by the next pass
+    }
+    T = prefix;
+    rem = remaining;
+}
+
+// The k-th largest of v[0..C) (1 <= k <= C) like sel_radix, in one histogram
+// pass when the values are spread: 2048 bins over [min, max] of the values
+// find the bin holding the k-th largest; when that bin holds at most 32
+// values one warp sorts them, otherwise sel_radix finishes inside the bin.
+__device__ __forceinline__ void sel_fine(const uint32_t* v, int C, int k, int* hist, int2* warp_tot, int* sh,
+                                         uint32_t& T, int& rem, int& eq) {
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    __shared__ uint32_t s_lo[kSelWarps], s_hi[kSelWarps], small[33];
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (int i = tid; i < C; i += kSelThreads) { lo = min(lo, v[i]); hi = max(hi, v[i]); }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) { s_lo[wid] = lo; s_hi[wid] = hi; }
+    for (int i = tid; i < 2048; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) { lo = min(lo, s_lo[w]); hi = max(hi, s_hi[w]); }
+    const uint32_t span = hi - lo;
+    const int shift = span < 2048u ? 0 : 21 - __clz(int(span));  // (span >> shift) < 2048
+    for (int i = tid; i < C; i += kSelThreads) atomicAdd(&hist[(v[i] - lo) >> shift], 1);
+    __syncthreads();
+    // thread t owns bins 2047-4t .. 2044-4t (counted from the top)
+    int loc[4], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) { loc[j] = hist[2047 - 4 * tid - j]; sum += loc[j]; }
+    const int2 inc = block_scan2<kSelThreads>(make_int2(sum, 0), warp_tot);
+    int above = inc.x - sum;
+    if (above < k && k <= inc.x) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (above < k && k <= above + loc[j]) { sh[0] = 2047 - 4 * tid - j; sh[1] = above; sh[2] = loc[j]; }
+            above += loc[j];
+        }
+    }
+    if (tid == 0) sh[3] = 0;
+    __syncthreads();
+    const int bin = sh[0], abv = sh[1], h = sh[2];
+    const int need = k - abv;                      // values to take from the bin
+    if (shift == 0) {                              // the bin is a single value
+        T = lo + uint32_t(bin);
+        rem = need;
+        eq = h;
+        return;
+    }
+    if (h > 32) {                                  // crowded bin: radix inside it
+        sel_radix(v, C, need, [&](int i) { return int((v[i] - lo) >> shift) == bin; }, hist, sh, T, rem, eq);
+        return;
+    }
+    // at most 32 values: gather them and let one warp sort them (descending)
+    for (int i = tid; i < C; i += kSelThreads)
+        if (int((v[i] - lo) >> shift) == bin) small[atomicAdd(&sh[3], 1)] = v[i];
+    __syncthreads();
+    if (wid == 0) {
+        uint32_t x = lane < h ? small[lane] : 0u;
+        // bitonic sort of 32 values, descending
+#pragma unroll
+        for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+            for (int st = size >> 1; st > 0; st >>= 1) {
+                const uint32_t y = __shfl_xor_sync(0xffffffffu, x, st);
+                const bool up = ((lane & size) == 0) == ((lane & st) == 0);
+                x = up ? max(x, y) : min(x, y);
+            }
+        }
+        const uint32_t t = __shfl_sync(0xffffffffu, x, need - 1);
+        const int gt = __popc(__ballot_sync(0xffffffffu, lane < h && x > t));
+        const int e = __popc(__ballot_sync(0xffffffffu, lane < h && x == t));
+        if (lane == 0) { small[32] = t; sh[1] = gt; sh[2] = e; }
+    }
+    __syncthreads();
+    T = small[32];
+    rem = need - sh[1];
+    eq = sh[2];
+    __syncthreads();
+}
+
+// Exact selection over a whole row in global memory by one CTA: three
+// histogram passes (11, 11 and 10 bits) and the ordered write.
+__device__ __noinline__ void sel_row_global(const float* s, int64_t n, int k, int32_t* out, int* hist,
+                                            int2* warp_tot, int* sh) {
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = k;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nbins = pass < 2 ? 2048 : 1024;
+        for (int i = tid; i < nbins; i += kSelThreads) hist[i] = 0;
+        __syncthreads();
+        for (int64_t i0 = 0; i0 < n; i0 += kSelThreads) {
+            const int64_t i = i0 + tid;
+            const uint32_t u = i < n ? order_key(s[i]) : 0u;
+            warp_hist_add(hist, i < n && (u & pmask) == prefix, (u >> shift) & uint32_t(nbins - 1));
+        }
+        __syncthreads();
+        // thread t owns bins nbins-1-4t .. nbins-4-4t (counted from the top)
+        int loc[4], sum = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int b = nbins - 1 - 4 * tid - j;
+            loc[j] = b >= 0 ? hist[b] : 0;
+            sum += loc[j];
+        }
+        const int2 inc = block_scan2<kSelThreads>(make_int2(sum, 0), warp_tot);
+        int above = inc.x - sum;
+        if (above < remaining && remaining <= inc.x) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (above < remaining && remaining <= above + loc[j]) {
+                    sh[0] = nbins - 1 - 4 * tid - j;
+                    sh[1] = above;
+                }
+                above += loc[j];
+            }
+        }
+        __syncthreads();
+        remaining -= sh[1];
+        prefix |= uint32_t(sh[0]) << shift;
+        pmask |= uint32_t(nbins - 1) << shift;
+        __syncthreads();
+    }
+    // every key above T = prefix, and the first `remaining` keys equal to it;
+    // warp w walks a contiguous segment of the row
+    const uint32_t T = prefix;
+    const int64_t seg = ((n + kSelWarps - 1) / kSelWarps + 31) / 32 * 32;
+    const int64_t lo = min(n, wid * seg), hi = min(n, lo + seg);
+    int gt = 0, eq = 0;
+    for (int64_t b0 = lo; b0 < hi; b0 += 32) {
+        const int64_t i = b0 + lane;
+        const uint32_t u = i < hi ? order_key(s[i]) : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, i < hi && u > T));
+        eq += __popc(__ballot_sync(0xffffffffu, i < hi && u == T));
+    }
+    const int2 incl = block_scan2<kSelThreads>(make_int2(lane == 0 ? gt : 0, lane == 0 ? eq : 0), warp_tot);
+    const int gt_incl = __shfl_sync(0xffffffffu, incl.x, 0), eq_incl = __shfl_sync(0xffffffffu, incl.y, 0);
+    int eq_before = eq_incl - eq;
+    int pos = (gt_incl - gt) + min(eq_before, remaining);
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int64_t b0 = lo; b0 < hi; b0 += 32) {
+        const int64_t i = b0 + lane;
+        const uint32_t u = i < hi ? order_key(s[i]) : 0u;
+        const bool is_eq = i < hi && u == T;
+        const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+        const int my_eq_rank = eq_before + __popc(eqm & lt_mask);
+        const bool take = i < hi && (u > T || (is_eq && my_eq_rank < remaining));
+        const unsigned tm = __ballot_sync(0xffffffffu, take);
+        if (take) {
+            const int p = pos + __popc(tm & lt_mask);
+            if (p < k) out[p] = int32_t(i);
+        }
+        pos += __popc(tm);
+        eq_before += __popc(eqm);
+    }
+}
+
+template <int CPR, int V>
+__global__ void __launch_bounds__(kSelThreads, 1)
+    topk_sel_kernel(const float* __restrict__ scores, int64_t ld, int64_t max_blocks,
+                    const int64_t* __restrict__ q_pos, int m, int W, int k, int32_t* __restrict__ idx,
+                    int seg, int cap, int vec) {
+    constexpr int kBatch = 4 * V * kSelThreads;     // keys of one batch of float4 chunks
+    extern __shared__ __align__(16) uint32_t dyn[];
+    uint32_t* ck = dyn;                  // leader: candidate keys [cap]
+    uint32_t* ci = dyn + cap;            // leader: candidate ids [cap]
+    uint32_t* bitmap = dyn + 2 * cap;    // leader: [ceil(max_blocks / 32)]
+    __shared__ int hist[2048];
+    __shared__ int2 warp_tot[32];
+    __shared__ int sh[4];
+    __shared__ int s_count;
+    __shared__ int s_bin[CPR];
+    pdl_wait();  // the scores come from the kernel before this one
+    pdl_launch_dependents();
+    const int tid = threadIdx.x, lane = tid & 31;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    int r = 0;
+    if constexpr (CPR > 1) r = int(cg::this_cluster().block_rank());
+    const int64_t row = blockIdx.x / CPR;
+    const float* s = scores + row * ld;
+    int32_t* out = idx + row * k;
+    const int n = int(min(n_elig(q_pos[row], m, W), max_blocks));
+    if (n <= k) {  // every eligible block is selected (uniform over the cluster)
+        if (r == 0)
+            for (int i = tid; i < k; i += kSelThreads) out[i] = i < n ? i : -1;
+        return;
+    }
+    if (r == 0 && tid == 0) s_count = 0;
+    if constexpr (CPR > 1) cluster_arrive_release();  // the leader's counter is set
+    int* lcount = &s_count;
+    uint32_t* lck = ck;
+    uint32_t* lci = ci;
+    int* lbin = s_bin;
+    if constexpr (CPR > 1) {
+        cg::cluster_group cl = cg::this_cluster();
+        lcount = cl.map_shared_rank(&s_count, 0);
+        lck = cl.map_shared_rank(ck, 0);
+        lci = cl.map_shared_rank(ci, 0);
+        lbin = cl.map_shared_rank(s_bin, 0);
+    }
+    const int base = r * seg, end = min(n, base + seg);
+    int b_r = 0;
+#pragma unroll 1
+    for (int b0 = base; b0 < end; b0 += kBatch) {
+        // this batch's keys (0 = no key: every real key is nonzero)
+        uint32_t key[4 * V];
+#pragma unroll
+        for (int u = 0; u < V; ++u) {
+            const int i0 = b0 + 4 * (u * kSelThreads + tid);
+            float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (vec && i0 + 3 < end) {
+                f = *reinterpret_cast<const float4*>(s + i0);
+            } else {
+                if (i0 < end) f.x = s[i0];
+                if (i0 + 1 < end) f.y = s[i0 + 1];
+                if (i0 + 2 < end) f.z = s[i0 + 2];
+                if (i0 + 3 < end) f.w = s[i0 + 3];
+            }
+            key[4 * u] = i0 < end ? order_key(f.x) : 0u;
+            key[4 * u + 1] = i0 + 1 < end ? order_key(f.y) : 0u;
+            key[4 * u + 2] = i0 + 2 < end ? order_key(f.z) : 0u;
+            key[4 * u + 3] = i0 + 3 < end ? order_key(f.w) : 0u;
+        }
+        if (b0 == base) {
+            // 1. the segment's threshold bin from its sample (the first chunk
+            // of every thread in the first batch)
+            if (n > kSelNoSampleMax) {
+                for (int i = tid; i < 2048; i += kSelThreads) hist[i] = 0;
+                __syncthreads();
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (key[c]) atomicAdd(&hist[key[c] >> 21], 1);
+                __syncthreads();
+                const int n_s = max(0, min(4 * kSelThreads, end - base));  // sampled keys
+                const float mean = float(k) * float(n_s) / float(n);
+                const int target = int(ceilf(mean + 4.f * sqrtf(mean))) + 16;
+                // thread t owns bins 2047-4t .. 2044-4t
+                int loc[4], sum = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) { loc[j] = hist[2047 - 4 * tid - j]; sum += loc[j]; }
+                const int2 inc = block_scan2<kSelThreads>(make_int2(sum, 0), warp_tot);
+                if (tid == 0) sh[3] = 0;
+                __syncthreads();
+                int above = inc.x - sum;
+                if (above < target && target <= inc.x) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (above < target && target <= above + loc[j]) sh[3] = 2047 - 4 * tid - j;
+                        above += loc[j];
+                    }
+                }
+                __syncthreads();
+                b_r = sh[3];  // 0 (every key) when the sample is short of the target
+            }
+            if constexpr (CPR > 1) cluster_wait_acquire();
+            else __syncthreads();
+        }
+        // 2. candidates into the leader: a per-warp count, one reservation per warp
+        int cnt = 0;
+#pragma unroll
+        for (int j = 0; j < 4 * V; ++j)
+            cnt += __popc(__ballot_sync(0xffffffffu, key[j] != 0u && int(key[j] >> 21) >= b_r));
+        int slot = 0;
+        if (lane == 0 && cnt) slot = atomicAdd(lcount, cnt);
+        slot = __shfl_sync(0xffffffffu, slot, 0);
+#pragma unroll
+        for (int j = 0; j < 4 * V; ++j) {
+            const bool c = key[j] != 0u && int(key[j] >> 21) >= b_r;
+            const unsigned bal = __ballot_sync(0xffffffffu, c);
+            if (c) {
+                const int p = slot + __popc(bal & lt_mask);
+                if (p < cap) {
+                    lck[p] = key[j];
+                    lci[p] = uint32_t(b0 + 4 * ((j >> 2) * kSelThreads + tid) + (j & 3));
+                }
+            }
+            slot += __popc(bal);
+        }
+    }
+    if (base >= end) {  // an empty segment still passes the barrier above
+        if constexpr (CPR > 1) cluster_wait_acquire();
+    }
+    if (tid == 0) lbin[r] = b_r;
+    if constexpr (CPR > 1) {
+        cg::this_cluster().sync();  // every candidate is in the leader
+        if (r != 0) return;
+    } else {
+        __syncthreads();
+    }
+    // 3. (leader) the k-th largest candidate; ties at T by the lowest ids
+    const int C = s_count;
+    uint32_t bmax = 0;
+#pragma unroll
+    for (int q = 0; q < CPR; ++q) bmax = max(bmax, uint32_t(s_bin[q]));
+    bool fast = C >= k && C <= cap;
+    uint32_t T = 0, T2 = 0;
+    int rem = 0, eq = 0;
+    if (fast) {
+        sel_fine(ck, C, k, hist, warp_tot, sh, T, rem, eq);
+        fast = T >= (bmax << 21);  // every key left out lies below T
+    }
+    if (!fast) {
+        sel_row_global(s, n, k, out, hist, warp_tot, sh);
+        return;
+    }
+    const bool all_eq = eq == rem;
+    if (!all_eq) {
+        // ck becomes 1 for keys above T, 0 below, ~id (>= 2^31) equal
+        for (int i = tid; i < C; i += kSelThreads) ck[i] = ck[i] == T ? ~ci[i] : (ck[i] > T ? 1u : 0u);
+        __syncthreads();
+        int r2, e2;
+        sel_radix(ck, C, rem, [&](int i) { return ck[i] > 1u; }, hist, sh, T2, r2, e2);
+    }
+    // 4. bitmap of the selected ids, then the ids in ascending order
+    const int words = (n + 31) >> 5;
+    for (int i = tid; i < words; i += kSelThreads) bitmap[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < C; i += kSelThreads) {
+        const bool take = all_eq ? ck[i] >= T : (ck[i] == 1u || (ck[i] > 1u && ck[i] >= T2));
+        if (take) atomicOr(&bitmap[ci[i] >> 5], 1u << (ci[i] & 31u));
+    }
+    __syncthreads();
+    const int per = (words + kSelThreads - 1) / kSelThreads;
+    const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+    int c = 0;
+    for (int wi = w0; wi < w1; ++wi) c += __popc(bitmap[wi]);
+    const int2 incl = block_scan2<kSelThreads>(make_int2(c, 0), warp_tot);
+    int pos = incl.x - c;
+    for (int wi = w0; wi < w1; ++wi) {
+        uint32_t b = bitmap[wi];
+        while (b) {
+            const int bit = __ffs(b) - 1;
+            b &= b - 1;
+            if (pos < k) out[pos] = wi * 32 + bit;
+            ++pos;
+        }
+    }
+}
+
+template <int CPR, int V>
+static cudaError_t launch_topk_sel(const float* scores, int64_t ld, int64_t max_blocks, const int64_t* q_pos,
+                                   int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s, bool pdl) {
+    // segment of each CTA: the row split in CPR parts, in whole float4 chunks of all threads
+    const int64_t unit = 4 * kSelThreads;
+    const int seg = int(ceil_div(ceil_div(max_blocks, CPR), unit) * unit);
+    const int cap = int(std::min<int64_t>(kSelCap, ceil_div(max_blocks, 4) * 4));
+    const size_t sm = (2 * size_t(cap) + size_t((max_blocks + 31) / 32)) * 4;
+    cudaError_t e = ensure_smem(topk_sel_kernel<CPR, V>, sm);
+    if (e != cudaSuccess) return e;
+    const int vec = ((reinterpret_cast<uintptr_t>(scores) & 15) == 0 && (ld % 4) == 0) ? 1 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(rows * CPR));
+    cfg.blockDim = dim3(kSelThreads);
+    cfg.dynamicSmemBytes = sm;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (CPR > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = CPR;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = na ? attr : nullptr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, topk_sel_kernel<CPR, V>, scores, ld, max_blocks, q_pos, m, W, k, idx, seg,
+                              cap, vec);
+}
+
 template <int E>
 static cudaError_t launch_topk_cluster(const float* scores, int64_t ld, int64_t max_blocks,
                                        const int64_t* q_pos, int m, int W, int k, int64_t rows,
@@ -401,7 +874,16 @@ static cudaError_t launch_topk_cluster(const float* scores, int64_t ld, int64_t 
 cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, const int64_t* q_pos,
                         int m, int W, int k, int64_t rows, int32_t* idx, cudaStream_t s, bool pdl) {
     if (rows == 0) return cudaSuccess;
-    // Few rows cannot fill the GPU with one CTA each: give each row a cluster.
+    // Sampled-threshold selection: one CTA per row for rows of up to 8,192
+    // scores (prefill chunks); for longer rows a cluster of 4 CTAs (up to 32K
+    // scores) or 8 CTAs per row, so that few rows still spread over many SMs.
+    if (k <= kSelCap / 2 && rows * 8 <= INT32_MAX && max_blocks <= INT32_MAX / 2) {
+        if (max_blocks <= 2048) return launch_topk_sel<1, 1>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
+        if (max_blocks <= 8192) return launch_topk_sel<1, 4>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
+        if (max_blocks <= 32768) return launch_topk_sel<4, 4>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
+        return launch_topk_sel<8, 8>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
+    }
+    // Few longer rows cannot fill the GPU with one CTA each: give each row a cluster.
     if (rows <= 2 * kNumSMs / kClu && k <= kClu * kCluThreads && max_blocks <= kClu * kCluThreads * 72) {
         const int64_t per = ceil_div(max_blocks, kClu * kCluThreads);
         if (per <= 2) return launch_topk_cluster<2>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);

@@ -17,13 +17,24 @@ from __future__ import annotations
 
 from dataclasses import dataclass
 
-from . import (BF16, FP8_S64, MXFP4, OP_DECODE, OP_HCA_ATTN, OP_PREFILL, Params, csa_compress,
-               csa_decode, csa_prefill, csa_workspace_size, empty_stored, hca_attn)
+from . import (BF16, FP8_S64, MXFP4, OP_DECODE, OP_HCA_ATTN, OP_PREFILL, OP_WINDOW_ATTN, Params,
+               csa_compress, csa_decode, csa_prefill, csa_workspace_size, empty_stored, hca_attn,
+               window_attn)
+
+
+def v4_pro_schedule(n_layers: int = 61, mtp: bool = True) -> list:
+    """Attention kind of each layer of DeepSeek-V4-Pro ("DeepSeek-V4 發佈說明",
+    section 架構實現: 61 layers; layers 0-1 use HCA, layers 2-60 alternate
+    between CSA and HCA, and the final MTP block uses only sliding-window
+    attention).  The alternation is read as starting with CSA at layer 2, the
+    order the note names them in; the MTP block is appended as a 62nd entry."""
+    kinds = ["hca" if i < 2 else ("csa" if (i - 2) % 2 == 0 else "hca") for i in range(n_layers)]
+    return kinds + (["window"] if mtp else [])
 
 
 @dataclass
 class LayerSpec:
-    kind: str          # "csa" | "hca"
+    kind: str          # "csa" | "hca" | "window" (the MTP block: sliding window only)
     p: Params          # m, window, top_k, heads, dims, scale, formats
     prior_tokens: int  # tokens already pooled into the cache (a multiple of m)
     new_tokens: int    # capacity for tokens appended after the prior cache
@@ -39,7 +50,8 @@ class Layer:
         p = spec.p
         self.m, self.W, self.d = p.m, p.window, p.head_dim
         self.cap_blocks = (spec.prior_tokens + spec.new_tokens) // self.m
-        self.kv = empty_stored(FP8_S64, self.cap_blocks, self.d, device)
+        # the window-only block keeps no pooled cache
+        self.kv = empty_stored(FP8_S64, self.cap_blocks, self.d, device) if spec.kind != "window" else None
         self.kI = empty_stored(MXFP4, self.cap_blocks, p.idx_dim, device) if spec.kind == "csa" else None
         # raw window: the W - 1 tokens before the first new token, then the new tokens
         self.raw_pos0 = spec.prior_tokens - (self.W - 1) if self.W > 0 else spec.prior_tokens
@@ -54,7 +66,7 @@ class Layer:
         self.t_next = spec.prior_tokens  # position of the next new token
         self._pooled = (spec.prior_tokens + self.m - 1) // self.m
         # decode workspace, allocated once so that decode steps can be captured in a graph
-        op = OP_DECODE if spec.kind == "csa" else OP_HCA_ATTN
+        op = {"csa": OP_DECODE, "hca": OP_HCA_ATTN, "window": OP_WINDOW_ATTN}[spec.kind]
         self.ws = torch.empty(csa_workspace_size(p, op, 1, 1, self.cap_blocks), dtype=torch.uint8,
                               device=device)
 
@@ -64,6 +76,8 @@ class Layer:
     def _pool_completed(self, t_end, bias, biasI):
         """Pool every block that completes at or before position t_end - 1 and
         has not been pooled yet."""
+        if self.kv is None:
+            return
         m, d = self.m, self.d
         for j in range(self._pooled, t_end // m):
             r0 = self._row(j * m)
@@ -104,9 +118,11 @@ class Layer:
         if spec.kind == "csa":
             csa_decode(p, 1, q, qI, w, self.kv, self.kI, self.cap_blocks, self.x, self.n_raw,
                        self.pos0, q_pos, sinks, out, idx_out, self.ws)
-        else:
+        elif spec.kind == "hca":
             hca_attn(p, 1, 1, q, self.kv, self.cap_blocks, self.x, self.n_raw, self.pos0, q_pos,
                      sinks, out, self.ws)
+        else:
+            window_attn(p, 1, 1, q, self.x, self.n_raw, self.pos0, q_pos, sinks, out, self.ws)
         self._pool_completed(t + 1, bias, biasI)
 
     def state(self):
@@ -140,6 +156,11 @@ class Layer:
             csa_prefill(p, 1, T, t0, self.x[rs:], self.n_raw - rs, rp0, self.z[r0:r0 + T],
                         bias, q, qI, w, self.kv, self.kI, self.cap_blocks, sinks, out, idx_out, ws)
             self._pooled = (t0 + T) // self.m
+        elif spec.kind == "window":
+            q_pos = torch.arange(t0, t0 + T, dtype=torch.int64, device=q.device)
+            ws = torch.empty(csa_workspace_size(p, OP_WINDOW_ATTN, 1, T, 0), dtype=torch.uint8,
+                             device=q.device)
+            window_attn(p, 1, T, q, self.x, self.n_raw, self.pos0, q_pos, sinks, out, ws)
         else:
             csa_compress(p, self.d, self.x[r0:r0 + n_pool], self.z[r0:r0 + n_pool], bias, n_pool,
                          _rows(self.kv, t0 // self.m, nb))

@@ -83,7 +83,25 @@ typedef struct csa_params {
     int32_t act_fmt;
     int32_t kv_fmt;
     int32_t idx_fmt;
+    uint32_t flags;    /* CSA_FLAG_* bits; 0 for the default behaviour */
 } csa_params;
+
+/* Flags of csa_params.
+ *
+ * CSA_FLAG_BATCH_INVARIANT -- batch-invariant, deterministic results ([WK]
+ *   基础设施: a batch-invariant, deterministic kernel library gives bitwise
+ *   reproducible inference).  Every output row is computed with the same
+ *   arithmetic in the same order whatever else is in the call: how a row's
+ *   attention items are split over CTAs, and the order in which the partial
+ *   results are combined, depend only on that row's own item count (about
+ *   three 64-item tiles per split, at most 8 splits), never on the number of
+ *   rows.  The indexer scores and the top-k selection are batch-invariant in
+ *   both modes (each score is one fixed-order sum; the selection is exact).
+ *   Without the flag the split count also depends on the number of rows, to
+ *   fill the GPU, so a row's output may differ in its last bits between
+ *   batch sizes (always within the matching tolerance).  Results are
+ *   deterministic run to run in both modes. */
+#define CSA_FLAG_BATCH_INVARIANT 0x1u
 
 /* ------------------------------------------------------------------------
  * csa_compress -- softmax-gated pooling with a learned positional bias
@@ -183,6 +201,19 @@ int hca_attn(const csa_params* p, int32_t batch, int32_t n_q, const void* q, con
              void* workspace, size_t ws_bytes, csa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * window_attn -- attention over the sliding window and the sink alone, with
+ * no pooled entry ([RN] 架構實現: the final MTP block of V4-Pro uses only
+ * sliding-window attention).  For query (b,i) at t = q_pos[b][i], over the
+ * raw tokens at positions t-W < pos <= t that lie in the raw buffer, the
+ * same softmax as sparse_mqa_attn with the sink in the denominator.
+ * Arguments as hca_attn without kv; p->m, p->top_k and p->kv_fmt are not used.
+ *   workspace: >= csa_workspace_size(p, CSA_OP_WINDOW_ATTN, batch, n_q, 0)
+ * ------------------------------------------------------------------------ */
+int window_attn(const csa_params* p, int32_t batch, int32_t n_q, const void* q, const void* raw,
+                int64_t n_raw, const int64_t* raw_pos0, const int64_t* q_pos, const float* sinks,
+                void* out, void* workspace, size_t ws_bytes, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * csa_decode -- one CSA read step for one new token per sequence:
  * indexer_score -> topk_select -> sparse_mqa_attn, launched back to back on
  * `stream` with the scores and selection in the workspace.  Shapes as above
@@ -226,6 +257,7 @@ int csa_prefill(const csa_params* p, int32_t batch, int64_t T, int64_t t0, const
 #define CSA_OP_HCA_ATTN 1
 #define CSA_OP_DECODE 2
 #define CSA_OP_PREFILL 3
+#define CSA_OP_WINDOW_ATTN 4
 
 /* Bytes of workspace an operation needs (0 on bad arguments; SIZE_MAX when
  * the size does not fit in size_t, which no buffer satisfies).  n_ctx is

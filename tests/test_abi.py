@@ -26,8 +26,8 @@ def _declared():
 
 def test_header_declares_the_entry_points():
     want = {"csa_compress", "csa_quantize", "indexer_score", "topk_select", "sparse_mqa_attn",
-            "hca_attn", "csa_decode", "csa_prefill", "csa_workspace_size", "csa_device_status",
-            "csa_strerror", "csa_version"}
+            "hca_attn", "window_attn", "csa_decode", "csa_prefill", "csa_workspace_size",
+            "csa_device_status", "csa_strerror", "csa_version"}
     assert want <= _declared()
 
 
@@ -132,9 +132,11 @@ def test_empty_inputs_are_no_ops_without_a_gpu():
                            fake, fake, fake, fake, fake, 1 << 30, fake, fake, fake, fake,
                            1 << 40, None) in (-1, -3, -4)
     # workspace queries for empty batches plan no split (this once divided by zero)
-    for op in (K.OP_DECODE, K.OP_PREFILL, K.OP_SPARSE_ATTN, K.OP_HCA_ATTN):
+    for op in (K.OP_DECODE, K.OP_PREFILL, K.OP_SPARSE_ATTN, K.OP_HCA_ATTN, K.OP_WINDOW_ATTN):
         assert 0 < lib.csa_workspace_size(P, op, 0, 1, 32768) < (1 << 20)
         assert 0 < lib.csa_workspace_size(P, op, 3, 0, 32768) < (1 << 20)
+    assert lib.window_attn(P, 0, 1, fake, fake, 8, fake, fake, None, fake, fake, 1 << 20, None) == 0
+    assert lib.window_attn(P, 2, 0, fake, fake, 8, fake, fake, None, fake, fake, 1 << 20, None) == 0
 
 
 def test_cuda_core_paths_refuse_more_rows_than_the_grid_holds():
@@ -147,3 +149,34 @@ def test_cuda_core_paths_refuse_more_rows_than_the_grid_holds():
     assert lib.sparse_mqa_attn(P, 2, 40000, fake, fake, None, 100, fake, fake, 8, fake, fake, None,
                                fake, fake, 1 << 40, None) == -3
     assert lib.indexer_score(P, 2, 40000, fake, None, fake, fake, None, 100, fake, fake, 100, None) == -3
+
+
+def test_window_attn_and_flags_host_errors():
+    lib = K.lib()
+    p = K.params(4, 128, 512, 64, 512, 64, 128, 0.044)
+    P = C.byref(p)
+    fake, odd = C.c_void_p(0x1000), C.c_void_p(0x1001)
+    # no query, no positions, a raw buffer without data, a misaligned output
+    assert lib.window_attn(P, 1, 1, None, fake, 8, fake, fake, None, fake, fake, 1 << 20, None) == -1
+    assert lib.window_attn(P, 1, 1, fake, fake, 8, fake, None, None, fake, fake, 1 << 20, None) == -1
+    assert lib.window_attn(P, 1, 1, fake, None, 8, fake, fake, None, fake, fake, 1 << 20, None) == -1
+    assert lib.window_attn(P, 1, 1, fake, fake, 8, fake, fake, None, odd, fake, 1 << 20, None) == -2
+    # a workspace below the plan (32 rows of a 128-token window split in two)
+    need = lib.csa_workspace_size(P, K.OP_WINDOW_ATTN, 32, 1, 0)
+    assert need > 32 * 64 * 512 * 4
+    assert lib.window_attn(P, 32, 1, fake, fake, 128, fake, fake, None, fake, fake, 16, None) == -4
+    # unknown flag bits are refused
+    bad = K.params(4, 128, 512, 64, 512, 64, 128, 0.044, flags=0x80)
+    assert lib.hca_attn(C.byref(bad), 1, 1, fake, fake, fake, 10, fake, 8, fake, fake, None,
+                        fake, fake, 1 << 20, None) == -1
+
+
+def test_batch_invariant_plan_depends_on_the_row_only():
+    """With CSA_FLAG_BATCH_INVARIANT the attention workspace grows exactly in
+    proportion to the rows (the split count per row is fixed), while the
+    default plan splits few rows more finely than many."""
+    inv = K.params(4, 128, 512, 64, 512, 64, 128, 0.044, flags=K.FLAG_BATCH_INVARIANT)
+    dft = K.params(4, 128, 512, 64, 512, 64, 128, 0.044)
+    ws = lambda p, b: K.csa_workspace_size(p, K.OP_SPARSE_ATTN, b, 1, 0) - 256
+    assert ws(inv, 32) == 32 * ws(inv, 1)
+    assert ws(dft, 1) > ws(dft, 32) / 32

@@ -392,3 +392,42 @@ def test_mxfp4_indexer_exact_across_block_exponents():
                    np.linalg.norm(kdq[:ne], axis=1)[None, :]).sum(0)
             err = np.abs(got[b, i, :ne] - ref[i, :ne])
             assert (err <= 1e-5 * mag + 1e-30).all(), (b, i, err.max())
+
+
+# Window-only attention (the MTP block): few-item rows (t < W) in one sequence,
+# full windows in the other, with and without sink-dominant logits; the bf16
+# tensor-core path and the fp32 CUDA-core path.
+@pytest.mark.parametrize("act,H,d,W,sink_shift", [
+    ("bf16", 64, 512, 128, None),
+    ("bf16", 64, 512, 128, 2.0),
+    ("f32", 8, 64, 64, None),
+])
+def test_window_attn_matches_oracle(act, H, d, W, sink_shift):
+    seed, batch = 41, 2
+    scale = 1 / math.sqrt(d)
+    q_pos = np.array([[0, 1, 4, 17, 60, W - 1], [W + 300, W + 301, W + 350, W + 400, W + 433, W + 439]],
+                     np.int64)
+    n_q = q_pos.shape[1]
+    raw_pos0 = np.array([0, W + 300 - W + 1], np.int64)
+    n_raw = int(max(q_pos[b].max() - raw_pos0[b] + 1 for b in range(batch)))
+    qv = synth.tensor_np(seed, "wq", (batch, n_q, H, d), dtype=act)
+    raw = synth.tensor_np(seed, "wraw", (batch, n_raw, d), dtype=act)
+    empty = oracle.Stored(oracle.F32, np.zeros((0, d), np.float32))
+    orc_in = [(act_orc(qv[b], act), empty, None, act_orc(raw[b], act), int(raw_pos0[b])) for b in range(batch)]
+    sinks = synth.tensor_np(seed, "wsink", (H,))
+    if sink_shift is not None:
+        sinks = np.max([sink_dominant(*orc_in[b], q_pos[b], H, 4, W, scale, sink_shift)
+                        for b in range(batch)], axis=0)
+    p = K.params(4, W, 1, H, d, 1, 32, scale, act_fmt=FMT[act], kv_fmt=FMT[act] if act == "f32" else K.FP8_S64)
+    out = torch.empty((batch, n_q, H, d), dtype=torch.float32 if act == "f32" else torch.bfloat16, device="cuda")
+    ws = torch.empty(K.csa_workspace_size(p, K.OP_WINDOW_ATTN, batch, n_q, 0), dtype=torch.uint8, device="cuda")
+    K.window_attn(p, batch, n_q, act_dev(qv, act), act_dev(raw, act), n_raw, up(raw_pos0), up(q_pos),
+                  up(sinks), out, ws)
+    got = down(out.float())
+    for b in range(batch):
+        ref = oracle.attention(*orc_in[b], sinks, q_pos[b], H, 4, W, scale)
+        if act == "f32":
+            assert_close_f32(got[b], ref, 1e-5, f"seq {b}")
+        else:
+            bound = attention_bound_stored(*orc_in[b], sinks, q_pos[b], H, 4, W, scale)
+            assert_attention_close(got[b], ref, bound, f"seq {b}")

@@ -203,3 +203,47 @@ def _run_hca(w, check_batches, draw_on_device=False):
         bound = attention_bound_stored(*args, sinks, [N], H, m, W, w.scale)[0]
         assert_attention_close(got[b], ref, bound, f"hca seq {b}")
     return got
+
+
+def test_batch_invariant_decode_is_bitwise_across_batch_sizes():
+    """With CSA_FLAG_BATCH_INVARIANT a sequence's selection and output bits do
+    not depend on the batch it is decoded in: the first sequence decoded
+    alone, in a batch of 8 and in a batch of 32 gives identical bytes (and the
+    first 8 agree between 8 and 32); parity with the oracle holds as usual."""
+    w = WORKLOADS["csa_decode_128k_b32"].with_(batch=32, n_ctx=16384, seed=15)
+    B, H, d, HI, dI, m, W, k = w.batch, w.H, w.d, w.HI, w.dI, w.m, w.W, w.k
+    nb = w.n_blocks
+    p = K.params(m, W, k, H, d, HI, dI, w.scale, FMT[w.act], FMT[w.kv], FMT[w.idx],
+                 flags=K.FLAG_BATCH_INVARIANT)
+    vals = {n: draw_np(w, n) for n in ("q", "qI", "w", "kv", "kI", "window", "sinks")}
+    kv_d, _ = both_stored(vals["kv"].reshape(-1, d), w.kv)
+    kI_d, _ = both_stored(vals["kI"].reshape(-1, dI), w.idx)
+    qI_d, _ = both_stored(vals["qI"].reshape(-1, dI), w.idx)
+    rng = np.random.default_rng(15)
+    q_pos = np.sort(rng.integers(3000, w.n_ctx + 1, size=B)).astype(np.int64)[::-1].copy()
+    q_pos[0] = w.n_ctx
+    q_d, win_d = act_dev(vals["q"], w.act), act_dev(vals["window"], w.act)
+    w_d, pos_d, pos0_d, sinks_d = up(vals["w"]), up(q_pos), up(q_pos - W + 1), up(vals["sinks"])
+    outs, sels = {}, {}
+    for b in (1, 8, 32):
+        sub = lambda st, per: K.Stored(st.fmt, st.data[:b * per], None if st.scales is None else st.scales[:b * per])
+        out = torch.empty((b, H, d), dtype=torch.bfloat16, device="cuda")
+        sel = torch.empty((b, k), dtype=torch.int32, device="cuda")
+        ws = torch.empty(K.csa_workspace_size(p, K.OP_DECODE, b, 1, nb), dtype=torch.uint8, device="cuda")
+        K.csa_decode(p, b, q_d[:b], sub(qI_d, HI), w_d[:b], sub(kv_d, nb), sub(kI_d, nb), nb, win_d[:b], W,
+                     pos0_d[:b], pos_d[:b], sinks_d, out, sel, ws)
+        outs[b], sels[b] = down(out), down(sel)
+    for b in (8, 32):
+        assert np.array_equal(sels[b][:1], sels[1]) and np.array_equal(outs[b][:1], outs[1]), f"batch {b}"
+    assert np.array_equal(sels[32][:8], sels[8]) and np.array_equal(outs[32][:8], outs[8])
+    # parity of the invariant mode (first sequence)
+    t = int(q_pos[0])
+    kv_o, kI_o = orc_quantize(vals["kv"][0], w.kv), orc_quantize(vals["kI"][0], w.idx)
+    scores = oracle.indexer(orc_quantize(vals["qI"][0].reshape(-1, dI), w.idx), vals["w"][0][None], kI_o, [t],
+                            HI, m, W)[0]
+    check_selection(sels[1][0], scores, min(oracle.n_elig(t, m, W), nb), k, what="seq 0")
+    args = (act_orc(vals["q"][0], w.act), kv_o, sels[1][:1], act_orc(vals["window"][0], w.act), t - W + 1)
+    ref = oracle.attention(*args, vals["sinks"], [t], H, m, W, w.scale)[0]
+    bound = attention_bound_stored(*args, vals["sinks"], [t], H, m, W, w.scale)[0]
+    got = synth.bf16_bits_to_f32_np(outs[1][0])
+    assert_attention_close(got, ref, bound, "seq 0")

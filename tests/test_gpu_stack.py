@@ -71,12 +71,13 @@ def _run_layer(kind, g, prior, chunk, steps, topk):
     """Run one layer (prior cache, chunk, decode steps) on the device; returns
     the outputs and selections of the chunk and of the decode steps, and the
     layer's caches."""
-    m = 4 if kind == "csa" else 128
+    m = 128 if kind == "hca" else 4
     p = K.params(m, W, topk if kind == "csa" else 1, H, D, HI, DI, SCALE, K.BF16, K.FP8_S64, K.MXFP4)
     n_new = chunk + steps
     L = Layer(LayerSpec(kind, p, prior, n_new))
-    K.csa_quantize(g("prior_kv", (prior // m, D)), K.Stored(K.FP8_S64, L.kv.data[:prior // m],
-                                                            L.kv.scales[:prior // m]))
+    if kind != "window":
+        K.csa_quantize(g("prior_kv", (prior // m, D)), K.Stored(K.FP8_S64, L.kv.data[:prior // m],
+                                                                L.kv.scales[:prior // m]))
     L.set_prior_window(g("x_prior", (W - 1, D), dt="bf16"))
     x, z = g("x", (n_new, D), dt="bf16"), g("z", (n_new, D), dt="bf16")
     bias, q, sinks = g("bias", (m, D), 0.1), g("q", (n_new, H, D), dt="bf16"), g("sinks", (H,))
@@ -102,7 +103,7 @@ def _run_layer(kind, g, prior, chunk, steps, topk):
     torch.cuda.synchronize()
     assert K.csa_device_status(reset=True) == 0
     res = dict(out=out, sel=sel, m=m, pooled=L._pooled,
-               kv=K.Stored(K.FP8_S64, down(L.kv.data), down(L.kv.scales)))
+               kv=None if L.kv is None else K.Stored(K.FP8_S64, down(L.kv.data), down(L.kv.scales)))
     if csa:
         res["kI"] = K.Stored(K.MXFP4, down(L.kI.data), down(L.kI.scales))
     return res
@@ -113,6 +114,8 @@ def _oracle_caches(kind, g, res, prior, n_pooled_new):
     pooling + quantisation of the new tokens' complete blocks.  Also checks
     the library's pooled rows against them."""
     m = res["m"]
+    if kind == "window":   # the MTP block keeps no pooled cache
+        return dict(kv=oracle.Stored(oracle.FP8_S64, np.zeros((0, D), np.uint8), np.zeros((0, D // 64), np.float32)))
     first, last = prior // m, res["pooled"]
     assert last - first == n_pooled_new
     x, z = g.host("x"), g.host("z")
@@ -182,9 +185,10 @@ def test_interleaved_stack_with_incremental_pooling(chunks):
     prior, topk = 2048, 128
     csa_chunk, hca_chunk, steps = chunks
     K.csa_device_status(reset=True)
-    for li, kind in enumerate(["csa", "hca", "csa", "hca"]):
-        chunk = csa_chunk if kind == "csa" else hca_chunk
-        m = 4 if kind == "csa" else 128
+    # four layers CSA, HCA, CSA, HCA and the MTP block (window only)
+    for li, kind in enumerate(["csa", "hca", "csa", "hca", "window"]):
+        chunk = hca_chunk if kind == "hca" else csa_chunk
+        m = 128 if kind == "hca" else 4
         g = _Draw(f"stack/{kind}", 40 + li)
         res = _run_layer(kind, g, prior, chunk, steps, topk)
         caches = _oracle_caches(kind, g, res, prior, (chunk + steps) // m)

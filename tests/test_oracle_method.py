@@ -296,3 +296,22 @@ def test_csa_composes_its_steps(orc):
     sel2 = orc.topk(sc, [t], k, m, W)
     o2 = orc.attention(q, kv, sel2, win, pos0, sinks, [t], H, m, W, 0.125)
     assert np.array_equal(sel, sel2) and np.array_equal(o, o2)
+
+
+@pytest.mark.parametrize("t,W,raw_pos0", [(50, 16, 0), (50, 16, 40), (5, 16, 0), (0, 1, 0), (30, 64, 10)])
+def test_window_only_attention_against_sdpa(orc, t, W, raw_pos0):
+    """The MTP block's window-only attention (no pooled entry) is SDPA over the
+    raw tokens t-W < i <= t that the raw buffer holds, with the sink: the
+    oracle's attention with an empty entry table must equal it."""
+    rng = np.random.default_rng(100 + t + W + raw_pos0)
+    H, d, m = 3, 16, 4
+    raw = rng.standard_normal((t + 1 - raw_pos0, d)).astype(np.float32)
+    q = rng.standard_normal((H, d)).astype(np.float32)
+    sinks = rng.standard_normal(H).astype(np.float32)
+    scale = 1 / math.sqrt(d)
+    empty = F32(orc, np.zeros((0, d), np.float32))
+    o = orc.attention(F32(orc, q), empty, None, F32(orc, raw), raw_pos0, sinks, [t], H, m, W, scale)[0]
+    window = [i for i in range(raw_pos0, t + 1) if t - W < i <= t]
+    keys = raw[[i - raw_pos0 for i in window]].astype(np.float64)
+    ref = _sdpa_ref(q.astype(np.float64), keys, sinks, scale)
+    assert np.allclose(o, ref, rtol=1e-10, atol=1e-12)
