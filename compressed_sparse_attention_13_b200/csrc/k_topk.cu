@@ -395,8 +395,8 @@ __global__ void __cluster_dims__(kClu, 1, 1) __launch_bounds__(kCluThreads)
 // CPR CTAs per row (one CTA for short rows), CTA r holding keys [r SEG,
 // (r+1) SEG) of the row, SEG = 4 V kSelThreads, loaded as float4 chunks (chunk
 // u of thread t: keys 4 (u kSelThreads + t) .. + 3 of the segment).
-//  1. each CTA builds an 11-bit histogram of a sample of its keys (chunk 0 of
-//     every thread) and takes a threshold bin b_r such that, by a wide margin,
+//  1. each CTA builds a 13-bit histogram of a sample of its keys (the first
+//     two chunks of every thread) and takes a threshold bin b_r such that, by a wide margin,
 //     its segment's share of the row's top k lies in bins >= b_r (rows of at
 //     most 4096 keys take every key: b_r = 0);
 //  2. each CTA pushes its keys in bins >= b_r, as (key, id) pairs, into the
@@ -413,7 +413,10 @@ __global__ void __cluster_dims__(kClu, 1, 1) __launch_bounds__(kCluThreads)
 // exact radix select over the whole row in global memory instead.
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kSelCap = 8192;           // most candidates kept in the leader's shared memory
+constexpr int kSelCap = 16384;          // most candidates kept in the leader's shared memory
+constexpr int kSelBinBits = 13;         // threshold bins: the top 13 bits of the order key
+constexpr int kSelBins = 1 << kSelBinBits;
+constexpr int kSelBinShift = 32 - kSelBinBits;
 constexpr int kSelNoSampleMax = 4096;   // rows this short take every key as a candidate
 
 __device__ __forceinline__ void cluster_arrive_release() {
@@ -655,7 +658,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     uint32_t* ck = dyn;                  // leader: candidate keys [cap]
     uint32_t* ci = dyn + cap;            // leader: candidate ids [cap]
     uint32_t* bitmap = dyn + 2 * cap;    // leader: [ceil(max_blocks / 32)]
-    __shared__ int hist[2048];
+    __shared__ int hist[kSelBins];
     __shared__ int2 warp_tot[32];
     __shared__ int sh[4];
     __shared__ int s_count;
@@ -712,30 +715,32 @@ __global__ void __launch_bounds__(kSelThreads, 1)
             key[4 * u + 3] = i0 + 3 < end ? order_key(f.w) : 0u;
         }
         if (b0 == base) {
-            // 1. the segment's threshold bin from its sample (the first chunk
-            // of every thread in the first batch)
+            // 1. the segment's threshold bin from its sample (the first two
+            // chunks of every thread in the first batch)
+            constexpr int kSampleChunks = V < 2 ? V : 2;
+            constexpr int kPer = kSelBins / kSelThreads;   // bins per thread in the scan
             if (n > kSelNoSampleMax) {
-                for (int i = tid; i < 2048; i += kSelThreads) hist[i] = 0;
+                for (int i = tid; i < kSelBins; i += kSelThreads) hist[i] = 0;
                 __syncthreads();
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    if (key[c]) atomicAdd(&hist[key[c] >> 21], 1);
+                for (int c = 0; c < 4 * kSampleChunks; ++c)
+                    if (key[c]) atomicAdd(&hist[key[c] >> kSelBinShift], 1);
                 __syncthreads();
-                const int n_s = max(0, min(4 * kSelThreads, end - base));  // sampled keys
+                const int n_s = max(0, min(4 * kSampleChunks * kSelThreads, end - base));  // sampled keys
                 const float mean = float(k) * float(n_s) / float(n);
                 const int target = int(ceilf(mean + 4.f * sqrtf(mean))) + 16;
-                // thread t owns bins 2047-4t .. 2044-4t
-                int loc[4], sum = 0;
+                // thread t owns bins kSelBins-1-kPer t .. kSelBins-kPer-kPer t (from the top)
+                int loc[kPer], sum = 0;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) { loc[j] = hist[2047 - 4 * tid - j]; sum += loc[j]; }
+                for (int j = 0; j < kPer; ++j) { loc[j] = hist[kSelBins - 1 - kPer * tid - j]; sum += loc[j]; }
                 const int2 inc = block_scan2<kSelThreads>(make_int2(sum, 0), warp_tot);
                 if (tid == 0) sh[3] = 0;
                 __syncthreads();
                 int above = inc.x - sum;
                 if (above < target && target <= inc.x) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (above < target && target <= above + loc[j]) sh[3] = 2047 - 4 * tid - j;
+                    for (int j = 0; j < kPer; ++j) {
+                        if (above < target && target <= above + loc[j]) sh[3] = kSelBins - 1 - kPer * tid - j;
                         above += loc[j];
                     }
                 }
@@ -749,13 +754,13 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         int cnt = 0;
 #pragma unroll
         for (int j = 0; j < 4 * V; ++j)
-            cnt += __popc(__ballot_sync(0xffffffffu, key[j] != 0u && int(key[j] >> 21) >= b_r));
+            cnt += __popc(__ballot_sync(0xffffffffu, key[j] != 0u && int(key[j] >> kSelBinShift) >= b_r));
         int slot = 0;
         if (lane == 0 && cnt) slot = atomicAdd(lcount, cnt);
         slot = __shfl_sync(0xffffffffu, slot, 0);
 #pragma unroll
         for (int j = 0; j < 4 * V; ++j) {
-            const bool c = key[j] != 0u && int(key[j] >> 21) >= b_r;
+            const bool c = key[j] != 0u && int(key[j] >> kSelBinShift) >= b_r;
             const unsigned bal = __ballot_sync(0xffffffffu, c);
             if (c) {
                 const int p = slot + __popc(bal & lt_mask);
@@ -787,7 +792,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     int rem = 0, eq = 0;
     if (fast) {
         sel_fine(ck, C, k, hist, warp_tot, sh, T, rem, eq);
-        fast = T >= (bmax << 21);  // every key left out lies below T
+        fast = T >= (bmax << kSelBinShift);  // every key left out lies below T
     }
     if (!fast) {
         sel_row_global(s, n, k, out, hist, warp_tot, sh);
@@ -877,7 +882,10 @@ cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, con
     // Sampled-threshold selection: one CTA per row for rows of up to 8,192
     // scores (prefill chunks); for longer rows a cluster of 4 CTAs (up to 32K
     // scores) or 8 CTAs per row, so that few rows still spread over many SMs.
-    if (k <= kSelCap / 2 && rows * 8 <= INT32_MAX && max_blocks <= INT32_MAX / 2) {
+    // (many short rows -- a prefill chunk -- are faster with the whole row in
+    // one CTA's shared memory and no sampling: topk_smem_kernel below)
+    const bool many_short = rows >= 2 * kNumSMs && max_blocks <= 4096;
+    if (k <= kSelCap / 2 && rows * 8 <= INT32_MAX && max_blocks <= INT32_MAX / 2 && !many_short) {
         if (max_blocks <= 2048) return launch_topk_sel<1, 1>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
         if (max_blocks <= 8192) return launch_topk_sel<1, 4>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
         if (max_blocks <= 32768) return launch_topk_sel<4, 4>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);

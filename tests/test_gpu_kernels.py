@@ -211,11 +211,15 @@ def _attn_case(act, kvf, H, d, batch, n_q, n_ent, W, k, m, seed, scale):
 
 
 # 2 x 12 and 2 x 20 query rows split each row 6 and 3 ways on the tensor-core
-# path, where the splits of a row form a cluster and combine in the kernel;
-# 6 rows split 10 ways and use the separate combine kernel.
+# path, where the splits of a row form a cluster and combine in the kernel
+# (2 x 9, 2 x 10 and 2 x 13 rows: 8, 7 and 5 splits); 6 rows split 10 ways
+# and use the separate combine kernel.
 @pytest.mark.parametrize("act,kvf,H,d,n_q,n_ent,W,k,m", [
     ("f32", "f32", 8, 64, 20, 256, 64, 16, 4),
     ("bf16", "fp8", 64, 512, 3, 700, 128, 512, 4),
+    ("bf16", "fp8", 64, 512, 9, 700, 128, 512, 4),
+    ("bf16", "fp8", 64, 512, 10, 700, 128, 512, 4),
+    ("bf16", "fp8", 64, 512, 13, 700, 128, 512, 4),
     ("bf16", "fp8", 64, 512, 12, 700, 128, 512, 4),
     ("bf16", "fp8", 64, 512, 20, 400, 128, 256, 4),
     ("bf16", "bf16", 64, 512, 4, 300, 128, 64, 4),
