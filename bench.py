@@ -836,6 +836,62 @@ def bench_schedule(dev, flush, stream, hbm_peak, steps=8):
                          "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4)}}
 
 
+def run_case(name, reps=3):
+    """One small named workload, run `reps` times, for profiling a kernel
+    under ncu (the bench's own timed region is not involved).  Inputs are
+    seeded; device memory stays at a few GB at most."""
+    import torch
+
+    import compressed_sparse_attention_13_b200 as K
+    from synth import tensor_torch
+    from synth.workloads import WORKLOADS, draw_torch
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if name == "decode_128k_b32":       # indexer, top-k, sparse attention (one csa_decode)
+        w = WORKLOADS[WORKLOAD]
+        S = setup_csa_decode(w, dev)
+        fn = lambda: csa_decode_call(w, S)
+    elif name == "hca_1m_b8":           # HCA attention over 8 x 8192 FP8 entries (+ the split combine)
+        w = WORKLOADS["hca_decode_1m_b8"]
+        B, N, H, d, m, W = w.batch, w.n_ctx, w.H, w.d, w.m, w.W
+        nb = N // m
+        p = K.params(m, W, 1, H, d, 1, 32, w.scale, K.BF16, K.FP8_S64, K.MXFP4)
+        kv = K.empty_stored(K.FP8_S64, B * nb, d, device=dev)
+        K.csa_quantize(tensor_torch(0, "case/hca/kv", (B * nb, d), device=dev), kv)
+        q = tensor_torch(0, "case/hca/q", (B, H, d), dtype="bf16", device=dev)
+        win = tensor_torch(0, "case/hca/win", (B, W, d), dtype="bf16", device=dev)
+        sinks = tensor_torch(0, "case/hca/sinks", (H,), device=dev)
+        q_pos = torch.full((B,), N, dtype=torch.int64, device=dev)
+        out = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(K.csa_workspace_size(p, K.OP_HCA_ATTN, B, 1, nb), dtype=torch.uint8, device=dev)
+        fn = lambda: K.hca_attn(p, B, 1, q, kv, nb, win, W, q_pos - W + 1, q_pos, sinks, out, ws)
+    elif name == "pool_hca":            # pooling 8 x 65,536 bf16 tokens at m' = 128 into FP8 entries
+        B, N, d, m = 8, 65536, 512, 128
+        p = K.params(m, 128, 1, 64, d, 1, 32, 1.0, K.BF16, K.FP8_S64, K.MXFP4)
+        x = tensor_torch(0, "case/pool/x", (B * N, d), dtype="bf16", device=dev)
+        z = tensor_torch(0, "case/pool/z", (B * N, d), dtype="bf16", device=dev)
+        bias = tensor_torch(0, "case/pool/bias", (m, d), 0.1, device=dev)
+        kv = K.empty_stored(K.FP8_S64, B * N // m, d, device=dev)
+        fn = lambda: K.csa_compress(p, d, x, z, bias, B * N, kv)
+    elif name == "prefill_topk":        # top-k of the 8K bf16 prefill: 8192 rows of up to 2048 scores
+        w = WORKLOADS["csa_prefill_8k_bf16"]
+        T, nb = w.n_ctx, w.n_ctx // w.m
+        p = K.params(w.m, w.W, w.k, w.H, w.d, w.HI, w.dI, w.scale, K.BF16, K.BF16, K.BF16)
+        scores = tensor_torch(0, "case/topk/s", (T, nb), device=dev)
+        q_pos = torch.arange(T, dtype=torch.int64, device=dev)
+        sel = torch.empty(T, w.k, dtype=torch.int32, device=dev)
+        fn = lambda: K.topk_select(p, 1, T, scores, nb, nb, q_pos, sel)
+    else:
+        raise SystemExit(f"unknown case {name}")
+    torch.cuda.empty_cache()   # only the case's own tensors stay on the device
+    for _ in range(reps):
+        fn()
+    torch.cuda.synchronize()
+    assert K.csa_device_status(reset=True) == 0
+    print(json.dumps({"case": name, "reps": reps, "ok": True}))
+
+
 # ------------------------------------------------------------- CPU oracle
 def _oracle_sample(w, seqs):
     """Host inputs for the sampled sequences, quantised by the oracle."""
@@ -943,7 +999,12 @@ def main():
                     "hca, prefill, stack, schedule) and print their results, without the main line")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--case", default="", help="run one small named workload (decode_128k_b32, hca_1m_b8, "
+                    "pool_hca, prefill_topk) a few times, for profiling, and exit")
     args = ap.parse_args()
+    if args.case:
+        run_case(args.case)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -395,8 +395,9 @@ __global__ void __cluster_dims__(kClu, 1, 1) __launch_bounds__(kCluThreads)
 // CPR CTAs per row (one CTA for short rows), CTA r holding keys [r SEG,
 // (r+1) SEG) of the row, SEG = 4 V kSelThreads, loaded as float4 chunks (chunk
 // u of thread t: keys 4 (u kSelThreads + t) .. + 3 of the segment).
-//  1. each CTA builds a 13-bit histogram of a sample of its keys (the first
-//     two chunks of every thread) and takes a threshold bin b_r such that, by a wide margin,
+//  1. each CTA builds an 11-bit histogram (13 bits for rows beyond 32K) of a
+//     sample of its keys (the first chunk, or two, of every thread in its
+//     first batch) and takes a threshold bin b_r such that, by a wide margin,
 //     its segment's share of the row's top k lies in bins >= b_r (rows of at
 //     most 4096 keys take every key: b_r = 0);
 //  2. each CTA pushes its keys in bins >= b_r, as (key, id) pairs, into the
@@ -414,9 +415,10 @@ __global__ void __cluster_dims__(kClu, 1, 1) __launch_bounds__(kCluThreads)
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelCap = 16384;          // most candidates kept in the leader's shared memory
-constexpr int kSelBinBits = 13;         // threshold bins: the top 13 bits of the order key
-constexpr int kSelBins = 1 << kSelBinBits;
-constexpr int kSelBinShift = 32 - kSelBinBits;
+// Threshold bins: the top 11 bits of the order key for rows of up to 32K
+// scores, 13 bits (and a sample twice as large) for longer rows, whose
+// skewed score tails would otherwise put too many keys into the threshold bin.
+__host__ __device__ constexpr int sel_bin_bits(int CPR) { return CPR >= 8 ? 13 : 11; }
 constexpr int kSelNoSampleMax = 4096;   // rows this short take every key as a candidate
 
 __device__ __forceinline__ void cluster_arrive_release() {
@@ -654,11 +656,14 @@ __global__ void __launch_bounds__(kSelThreads, 1)
                     const int64_t* __restrict__ q_pos, int m, int W, int k, int32_t* __restrict__ idx,
                     int seg, int cap, int vec) {
     constexpr int kBatch = 4 * V * kSelThreads;     // keys of one batch of float4 chunks
+    constexpr int kSelBinBits = sel_bin_bits(CPR);
+    constexpr int kSelBins = 1 << kSelBinBits;
+    constexpr int kSelBinShift = 32 - kSelBinBits;
     extern __shared__ __align__(16) uint32_t dyn[];
     uint32_t* ck = dyn;                  // leader: candidate keys [cap]
     uint32_t* ci = dyn + cap;            // leader: candidate ids [cap]
     uint32_t* bitmap = dyn + 2 * cap;    // leader: [ceil(max_blocks / 32)]
-    __shared__ int hist[kSelBins];
+    __shared__ int hist[kSelBins > 2048 ? kSelBins : 2048];   // (sel_fine and the fallback use 2048)
     __shared__ int2 warp_tot[32];
     __shared__ int sh[4];
     __shared__ int s_count;
@@ -717,7 +722,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         if (b0 == base) {
             // 1. the segment's threshold bin from its sample (the first two
             // chunks of every thread in the first batch)
-            constexpr int kSampleChunks = V < 2 ? V : 2;
+            constexpr int kSampleChunks = (V < 2 || CPR < 8) ? 1 : 2;
             constexpr int kPer = kSelBins / kSelThreads;   // bins per thread in the scan
             if (n > kSelNoSampleMax) {
                 for (int i = tid; i < kSelBins; i += kSelThreads) hist[i] = 0;
