@@ -354,7 +354,8 @@ def run_ours(args):
         legs = {"hca": lambda: bench_hca(args, dev, flush, stream, hbm_peak),
                 "prefill": lambda: bench_prefill(dev, flush, stream, bf16_peak),
                 "stack": lambda: bench_stack(dev, flush, stream, hbm_peak, bf16_peak),
-                "schedule": lambda: bench_schedule(dev, flush, stream, hbm_peak)}
+                "schedule": lambda: bench_schedule(dev, flush, stream, hbm_peak),
+                "indexer": lambda: bench_indexer_variants(args, dev, flush, stream, hbm_peak)}
         print(json.dumps({n: legs[n]() for n in args.only_legs.split(",")}), flush=True)
         return
 
@@ -467,11 +468,17 @@ def run_ours(args):
         "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
     }
-    legs = set(args.legs.split(",")) if args.legs else {"hca", "prefill", "stack", "schedule"}
+    legs = set(args.legs.split(",")) if args.legs else {"hca", "indexer", "prefill", "stack", "schedule"}
     if world == 1 and rank == 0 and not args.no_extra:
         if "hca" in legs:
             result["hca_decode"] = bench_hca(args, dev, flush, stream, hbm_peak)
         del S
+        torch.cuda.empty_cache()
+        if "indexer" in legs:
+            try:
+                result["indexer_write_path"] = bench_indexer_variants(args, dev, flush, stream, hbm_peak)
+            except Exception as exc:  # an extra leg must not lose the main line
+                result["indexer_write_path"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
         torch.cuda.empty_cache()
         for key, name, leg in (("prefill_8k_bf16", "prefill", lambda: bench_prefill(dev, flush, stream, bf16_peak)),
                                ("stack_c4", "stack", lambda: bench_stack(dev, flush, stream, hbm_peak, bf16_peak)),
@@ -531,6 +538,54 @@ def bench_hca(args, dev, flush, stream, hbm_peak):
             "compress": {"workload": "pool 8 x 1M bf16 tokens at m'=128 -> FP8",
                          "ms": round(t_comp, 3), "bytes": comp_bytes,
                          "achieved_gbs": round(comp_bytes / (t_comp / 1e3) / 1e9, 1)}}
+
+
+def bench_indexer_variants(args, dev, flush, stream, hbm_peak):
+    """The indexer of the 128K x 32 decode step on its write-path variants,
+    each graph-replayed after an L2 flush: MXFP4 queries stored beforehand
+    (the default), the same with the separate fp32 -> MXFP4 quantise launch
+    in the step, bf16 queries quantised inside the indexer, and the exact
+    E2M1 -> E4M3 expansion on the MXFP8 MMA (alone and with bf16 queries)."""
+    import torch
+
+    import compressed_sparse_attention_13_b200 as K
+    from synth.workloads import WORKLOADS, draw_torch
+
+    w = WORKLOADS[WORKLOAD]
+    B, HI, dI, m, W = w.batch, w.HI, w.dI, w.m, w.W
+    nb = w.n_ctx // m
+    kv = draw_torch(w, "kI", device=dev).reshape(-1, dI)
+    kI = K.empty_stored(K.MXFP4, B * nb, dI, device=dev)
+    K.csa_quantize(kv, kI)
+    del kv
+    qf = draw_torch(w, "qI", device=dev).reshape(-1, dI).contiguous()
+    qb = qf.to(torch.bfloat16)
+    qs = K.empty_stored(K.MXFP4, B * HI, dI, device=dev)
+    wt = draw_torch(w, "w", device=dev)
+    q_pos = torch.full((B,), w.n_ctx, dtype=torch.int64, device=dev)
+    scores = torch.empty(B, nb, dtype=torch.float32, device=dev)
+    K.csa_quantize(qf, qs)
+    prm = lambda f: K.params(m, W, w.k, w.H, w.d, HI, dI, w.scale, K.BF16, K.FP8_S64, K.MXFP4, flags=f)
+    p0, pq, p8, pq8 = prm(0), prm(K.FLAG_QI_BF16), prm(K.FLAG_INDEXER_FP8), prm(K.FLAG_QI_BF16 | K.FLAG_INDEXER_FP8)
+    cases = {
+        "mxfp4_stored_query": lambda: K.indexer_score(p0, B, 1, qs, wt, kI, nb, q_pos, scores, nb),
+        "quantise_then_mxfp4": lambda: (K.csa_quantize(qf, qs),
+                                        K.indexer_score(p0, B, 1, qs, wt, kI, nb, q_pos, scores, nb)),
+        "mxfp4_bf16_query_fused": lambda: K.indexer_score(pq, B, 1, K.Stored(K.BF16, qb), wt, kI, nb, q_pos,
+                                                          scores, nb),
+        "fp8_expanded": lambda: K.indexer_score(p8, B, 1, qs, wt, kI, nb, q_pos, scores, nb),
+        "fp8_expanded_bf16_query": lambda: K.indexer_score(pq8, B, 1, K.Stored(K.BF16, qb), wt, kI, nb,
+                                                           q_pos, scores, nb),
+    }
+    n_vis = max(0, min((w.n_ctx - W) // m, nb))
+    key_bytes = B * n_vis * (dI // 2 + dI // 32)
+    res = {"workload": WORKLOAD, "key_bytes": key_bytes}
+    for name, fn in cases.items():
+        t = statistics.mean(time_steps(graphed(fn), args.steps, args.warmup, flush, stream))
+        res[name] = {"us": round(t * 1e3, 2), "key_gbs": round(key_bytes / (t / 1e3) / 1e9, 1),
+                     "frac": round(key_bytes / (t / 1e3) / 1e9 / hbm_peak, 4)}
+    assert K.csa_device_status(reset=True) == 0
+    return res
 
 
 def _causal_pairs(T, m, W, k, t0=0):
@@ -993,10 +1048,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true", help="skip the extra legs")
-    ap.add_argument("--legs", default="", help="extra legs to run, comma-separated among hca, prefill, "
+    ap.add_argument("--legs", default="", help="extra legs to run, comma-separated among hca, indexer, prefill, "
                     "stack, schedule (default: all)")
     ap.add_argument("--only-legs", default="", help="run only these extra legs (comma-separated among "
-                    "hca, prefill, stack, schedule) and print their results, without the main line")
+                    "hca, indexer, prefill, stack, schedule) and print their results, without the main line")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--case", default="", help="run one small named workload (decode_128k_b32, hca_1m_b8, "

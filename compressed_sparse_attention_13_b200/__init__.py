@@ -21,6 +21,8 @@ from dataclasses import dataclass
 F32, BF16, FP8_S64, MXFP4 = 0, 1, 2, 3
 OP_SPARSE_ATTN, OP_HCA_ATTN, OP_DECODE, OP_PREFILL, OP_WINDOW_ATTN = 0, 1, 2, 3, 4
 FLAG_BATCH_INVARIANT = 0x1
+FLAG_QI_BF16 = 0x2
+FLAG_INDEXER_FP8 = 0x4
 DEV_BAD_INDEX, DEV_RANGE, DEV_TIMEOUT = 0x1, 0x2, 0x4
 NOALLOC_SCRATCH_BYTES = 32 << 20   # CSA_NOALLOC_SCRATCH_BYTES
 ERR_WORKSPACE = -4

@@ -38,7 +38,7 @@ static bool idx_ok(int f) { return f == CSA_F32 || f == CSA_BF16 || f == CSA_MXF
 static int check_params(const csa_params* p, bool need_idx, bool need_attn) {
     if (!p) return CSA_ERR_ARG;
     if (p->m <= 0 || p->window < 0) return CSA_ERR_ARG;
-    if (p->flags & ~CSA_FLAG_BATCH_INVARIANT) return CSA_ERR_ARG;
+    if (p->flags & ~(CSA_FLAG_BATCH_INVARIANT | CSA_FLAG_QI_BF16 | CSA_FLAG_INDEXER_FP8)) return CSA_ERR_ARG;
     if (need_attn) {
         if (p->n_heads <= 0 || p->head_dim <= 0 || (p->head_dim % 64) != 0) return CSA_ERR_ARG;
         if (!act_ok(p->act_fmt) || !kv_ok(p->kv_fmt)) return CSA_ERR_ARG;
@@ -212,15 +212,21 @@ int indexer_score(const csa_params* p, int32_t batch, int32_t n_q, const void* q
     if (batch < 0 || n_q < 0 || max_blocks < 0 || ld_scores < max_blocks) return CSA_ERR_ARG;
     if (batch == 0 || n_q == 0 || max_blocks == 0) return CSA_OK;
     if (!qI || !w || !kI || !q_pos || !scores) return CSA_ERR_ARG;
-    if (p->idx_fmt == CSA_MXFP4 && (!qI_scales || !kI_scales)) return CSA_ERR_ARG;
+    // the write-path variants of the MXFP4 indexer (bf16 queries quantised in
+    // the kernel; the exact E2M1 -> E4M3 expansion on the MXFP8 MMA)
+    const bool q_bf16 = (p->flags & CSA_FLAG_QI_BF16) != 0;
+    const bool fp8 = (p->flags & CSA_FLAG_INDEXER_FP8) != 0;
+    if ((q_bf16 || fp8) && p->idx_fmt != CSA_MXFP4) return CSA_ERR_ARG;
+    if (p->idx_fmt == CSA_MXFP4 && ((!q_bf16 && !qI_scales) || !kI_scales)) return CSA_ERR_ARG;
     if (!aligned16(qI) || !aligned16(kI) || !aligned16(scores) || !aligned16(qI_scales) ||
         !aligned16(kI_scales))
         return CSA_ERR_ALIGN;
     if (indexer_tc_supported(p->idx_fmt, p->idx_heads, p->idx_dim, max_blocks, batch,
                              int64_t(batch) * n_q))
-        return cuda_status(launch_indexer_tc(qI, qI_scales, w, kI, kI_scales, max_blocks, q_pos,
-                                             batch, n_q, p->m, p->window, scores, ld_scores,
-                                             (cudaStream_t)stream));
+        return cuda_status(launch_indexer_tc(qI, q_bf16 ? nullptr : qI_scales, w, kI, kI_scales, max_blocks,
+                                             q_pos, batch, n_q, p->m, p->window, scores, ld_scores, q_bf16,
+                                             fp8, (cudaStream_t)stream));
+    if (q_bf16 || fp8) return CSA_ERR_UNSUPPORTED;  // the variants exist on the tensor-core path only
     if (indexer_bf16_tc_supported(p->idx_fmt, p->idx_heads, p->idx_dim, max_blocks, batch, n_q))
         return cuda_status(launch_indexer_bf16_tc(qI, w, kI, max_blocks, q_pos, batch, n_q, p->m,
                                                   p->window, scores, ld_scores, (cudaStream_t)stream));

@@ -67,6 +67,21 @@ __device__ __forceinline__ uint32_t f32_to_e2m1(float v) {
     return (uint32_t)__nv_cvt_float_to_fp4(v, __NV_E2M1, cudaRoundNearest) & 0xFu;
 }
 
+// Two fp32 values -> one byte of two E2M1 codes (lo in the low nibble), round
+// to nearest even, saturating to +-6.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+    uint16_t r;
+    asm("{ .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n mov.b16 %0, {t, 0}; }"
+        : "=h"(r)
+        : "f"(hi), "f"(lo));
+    return r & 0xFFu;
+}
+
+// 2^e as a float for e in [-127, 127] (exact).
+__device__ __forceinline__ float pow2f(int e) {
+    return e >= -126 ? __int_as_float((e + 127) << 23) : __int_as_float(0x00400000);
+}
+
 // floor(log2(a)) for a finite a > 0 (subnormals included).
 __device__ __forceinline__ int ilog2_floor(float a) {
     const uint32_t u = __float_as_uint(a);

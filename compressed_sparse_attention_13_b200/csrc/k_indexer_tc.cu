@@ -40,6 +40,8 @@
 // All waits are bounded (sm100::mbar_wait); after a timed-out wait a role
 // keeps iterating without waiting or touching memory, so every thread still
 // reaches the named and final barriers.
+#include <string.h>
+
 #include "kernels.h"
 #include "sm100.cuh"
 #include "tmap.h"
@@ -52,25 +54,39 @@ constexpr int kHI = 64, kDI = 128;
 constexpr int kTileKeys = 128;                         // keys per MMA (M)
 constexpr int kStepKeys = 128;                         // keys per pipeline step
 constexpr int kTilesPerStep = kStepKeys / kTileKeys;
-constexpr int kStages = 8;
 constexpr int kQBufs = 4, kAccBufs = 2;
 constexpr int kEpiGroups = 1;                          // epilogue groups of 4 warps
-constexpr int kCtasPerSm = 2;                          // two independent pipelines per SM
 constexpr int kKeyBytes = kDI / 2;                     // 64: packed E2M1
 constexpr int kAData = kStepKeys * kKeyBytes;          // 8192
 constexpr int kQData = kHI * kKeyBytes;                // 4096
+constexpr int kA8Data = kStepKeys * kDI;               // 16384: E4M3 keys of a step (FP8 variant)
+constexpr int kQ8Data = kHI * kDI;                     // 8192: E4M3 query block (FP8 variant)
 constexpr int kAccCols = kTilesPerStep * 64;           // tiles x 64 heads
-constexpr int kSfaPerStage = 8 * kTilesPerStep;        // two MMA k-steps x 4 columns per tile
-constexpr int kSfaCol = kAccBufs * kAccCols;           // 128
-constexpr int kSfbCol = kSfaCol + kSfaPerStage * kStages;  // 192: 4 columns per buffer
 constexpr int kTmemCols = 256;
 constexpr int kEpiWarp0 = 6;
-constexpr int kThreads = 32 * (kEpiWarp0 + 4 * kEpiGroups);
-static_assert(kSfbCol + 4 * kStages <= kTmemCols, "TMEM columns");
+constexpr int kConvWarp0 = kEpiWarp0 + 4 * kEpiGroups; // FP8 variant: E2M1 -> E4M3 converters
+
+// Per variant: the MXFP4 kernel (kind::mxf4, two E8M0 scales per row and
+// MMA, K = 64) runs two pipelines per SM with an 8-stage ring; the FP8
+// variant (kind::mxf8f6f4, one scale per row and MMA, K = 32) carries the
+// expanded E4M3 copies as well, so it runs one CTA per SM with a 4-stage ring.
+template <bool F8>
+struct Cfg {
+    static constexpr int kStages = F8 ? 4 : 8;
+    static constexpr int kCtasPerSm = F8 ? 1 : 2;
+    static constexpr int kThreads = 32 * (kConvWarp0 + (F8 ? 4 : 0));
+    static constexpr int kKSteps = F8 ? 4 : 2;                    // MMAs per 128-dim tile
+    static constexpr int kSfaPerStage = 4 * kKSteps * kTilesPerStep;  // 4 columns per k-step
+    static constexpr int kSfbPerBuf = 2 * kKSteps;                // 2 columns (64 heads) per k-step
+    static constexpr int kSfaCol = kAccBufs * kAccCols;           // 128
+    static constexpr int kSfbCol = kSfaCol + kSfaPerStage * kStages;
+    static_assert(kSfbCol + kSfbPerBuf * kStages <= kTmemCols, "TMEM columns");
+};
 
 struct IdxTcArgs {
     const uint8_t* kIs;   // [batch][max_blocks][4] E8M0
-    const uint8_t* qIs;   // [rows][64][4] E8M0
+    const uint8_t* qIs;   // [rows][64][4] E8M0 (stored MXFP4 queries)
+    const uint16_t* qraw; // [rows][64][128] bf16 (queries quantised in the kernel)
     const float* w;       // [rows][64]
     const int64_t* q_pos; // [rows]
     float* scores;        // [rows][ld]
@@ -79,13 +95,18 @@ struct IdxTcArgs {
     int64_t rows, tiles_per_row, units;
 };
 
+template <bool F8>
 struct Smem {
-    uint8_t a[kStages][kAData];        // 1024-aligned: key steps (64-byte swizzle)
+    static constexpr int kSt = Cfg<F8>::kStages;
+    uint8_t a[kSt][kAData];            // 1024-aligned: key steps (64-byte swizzle)
     uint8_t q[kQBufs][kQData];         // query blocks (64-byte swizzle)
-    uint32_t a_sf[kStages][kStepKeys]; // keys' four E8M0 bytes
+    uint8_t a8[F8 ? kSt : 1][F8 ? kA8Data : 1024];   // FP8 variant: E4M3 keys (128-byte swizzle)
+    uint8_t q8[F8 ? kQBufs : 1][F8 ? kQ8Data : 1024];  // FP8 variant: E4M3 query blocks
+    uint32_t a_sf[kSt][kStepKeys];     // keys' four E8M0 bytes
+    uint32_t q_sf[kQBufs][kHI];        // queries quantised here: their four E8M0 bytes per head
     float ew[kEpiGroups][kHI];         // per epilogue group: weights of its current row
-    uint64_t a_full[kStages], a_empty[kStages], sf_full[kStages];
-    uint64_t q_full[kQBufs], q_empty[kQBufs];
+    uint64_t a_full[kSt], a_empty[kSt], sf_full[kSt], a8_full[kSt];
+    uint64_t q_full[kQBufs], q_empty[kQBufs], q8_full[kQBufs];
     uint64_t acc_full[kAccBufs], acc_empty[kAccBufs];
     uint32_t tmem_base;
 };
@@ -133,21 +154,85 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
     return d;
 }
 
+
+// Four E2M1 codes (the low 16 bits, element i in nibble i) -> four E4M3
+// bytes.  Every E2M1 value (+-{0, 0.5, 1, 1.5, 2, 3, 4, 6}) is an E4M3
+// value, so the expansion is exact: a byte-table lookup on the magnitude
+// and the sign moved to bit 7.
+__device__ __forceinline__ uint32_t e4m3x4_of_e2m1x4(uint32_t x) {
+    uint32_t mag, sgn;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(mag) : "r"(0x3C383000u), "r"(0x4C484440u), "r"(x & 0x7777u));
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(sgn) : "r"(0x00008000u), "r"(0u), "r"((x >> 3) & 0x1111u));
+    return mag | sgn;
+}
+
+// One 64-byte-swizzled row of 128 packed E2M1 codes -> the same row as 128
+// E4M3 bytes in the 128-byte-swizzled K-major layout.
+__device__ __forceinline__ void expand_row(const uint8_t* src, uint8_t* dst, uint32_t row) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const uint4 w = *reinterpret_cast<const uint4*>(src + sm100::sw64_offset(row, c));
+        const uint4 lo = make_uint4(e4m3x4_of_e2m1x4(w.x), e4m3x4_of_e2m1x4(w.x >> 16),
+                                    e4m3x4_of_e2m1x4(w.y), e4m3x4_of_e2m1x4(w.y >> 16));
+        const uint4 hi = make_uint4(e4m3x4_of_e2m1x4(w.z), e4m3x4_of_e2m1x4(w.z >> 16),
+                                    e4m3x4_of_e2m1x4(w.w), e4m3x4_of_e2m1x4(w.w >> 16));
+        *reinterpret_cast<uint4*>(dst + sm100::sw128_offset(row, 2 * c)) = lo;
+        *reinterpret_cast<uint4*>(dst + sm100::sw128_offset(row, 2 * c + 1)) = hi;
+    }
+}
+
+// Quantise 32 bf16 values (one MXFP4 block) as csa_quantize does: block
+// exponent X = floor(log2(max |v|)) - 2 clamped to [-127, 127] (0 for an
+// all-zero block), codes = E2M1(v * 2^-X) rounded to nearest even.  Returns
+// the E8M0 byte X + 127; the 16 code bytes go to out.
+__device__ __forceinline__ uint32_t quant_block32(const uint4 (&v)[4], uint4& out) {
+    float f[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            f[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            f[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    int X = amax > 0.f ? ilog2_floor(amax) - 2 : 0;
+    X = max(-127, min(127, X));
+    const float inv = pow2f(-X);
+    uint32_t b[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) b[i] = cvt_e2m1x2(__fmul_rn(f[2 * i], inv), __fmul_rn(f[2 * i + 1], inv));
+    out = make_uint4(b[0] | b[1] << 8 | b[2] << 16 | b[3] << 24, b[4] | b[5] << 8 | b[6] << 16 | b[7] << 24,
+                      b[8] | b[9] << 8 | b[10] << 16 | b[11] << 24, b[12] | b[13] << 8 | b[14] << 16 | b[15] << 24);
+    return uint32_t(X + 127);
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+template <bool QRAW, bool F8>
+__global__ void __launch_bounds__(Cfg<F8>::kThreads, Cfg<F8>::kCtasPerSm)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_q, const IdxTcArgs a) {
+    using C = Cfg<F8>;
+    constexpr int kStages = C::kStages;
     extern __shared__ uint8_t smem_raw[];
-    Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem<F8>& S = *reinterpret_cast<Smem<F8>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     using namespace sm100;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&S.a_full[i], 1); mbar_init(&S.a_empty[i], 1); mbar_init(&S.sf_full[i], 4);  // one arrival per scale-writer warp
+            mbar_init(&S.a8_full[i], 4);  // one arrival per converter warp
         }
-        for (int i = 0; i < kQBufs; ++i) { mbar_init(&S.q_full[i], 1); mbar_init(&S.q_empty[i], 1); }
+        for (int i = 0; i < kQBufs; ++i) {
+            mbar_init(&S.q_full[i], QRAW ? 4 : 1);  // the tensor copy, or one arrival per quantiser warp
+            mbar_init(&S.q_empty[i], 1);
+            mbar_init(&S.q8_full[i], 4);
+        }
         for (int i = 0; i < kAccBufs; ++i) { mbar_init(&S.acc_full[i], 1); mbar_init(&S.acc_empty[i], 4); }
         fence_mbar_init();
     }
@@ -169,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             int64_t cur_row = -1;
             bool ok = true;
             for (int it = 0; ok && tw.next(a); ++it) {
-                if (tw.row != cur_row) {
+                if (!QRAW && tw.row != cur_row) {
                     cur_row = tw.row;
                     ++rc;
                     const int qb = rc & (kQBufs - 1);
@@ -204,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     } else if (warp == 1) {
         // --------------------------------------------------------------- MMA
         if (lane == 0) {
-            constexpr uint32_t idesc = instr_desc_mxf4(128, 64);
+            constexpr uint32_t idesc = F8 ? instr_desc_mxf8_e4m3(128, 64) : instr_desc_mxf4(128, 64);
             TileWalk tw(a, u0, u1);
             int64_t cur_row = -1;
             int rc = -1, st = 0;
@@ -216,26 +301,36 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     if (rc >= 0) mma_commit(&S.q_empty[rc & (kQBufs - 1)]);
                     cur_row = tw.row;
                     ++rc;
-                    ok = mbar_wait(&S.q_full[rc & (kQBufs - 1)], uint32_t(rc / kQBufs) & 1u);
+                    const uint32_t qpar = uint32_t(rc / kQBufs) & 1u;
+                    ok = mbar_wait(F8 ? &S.q8_full[rc & (kQBufs - 1)] : &S.q_full[rc & (kQBufs - 1)], qpar);
                 }
                 const int b = it % kAccBufs;
                 const uint32_t par = uint32_t(it / kAccBufs) & 1u;
-                if (ok) ok = mbar_wait(&S.a_full[st], ph);
+                if (ok) ok = mbar_wait(F8 ? &S.a8_full[st] : &S.a_full[st], ph);
                 if (ok) ok = mbar_wait(&S.sf_full[st], ph);
                 if (ok && it >= kAccBufs) ok = mbar_wait(&S.acc_empty[b], par ^ 1u);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(S.a[st]), b0 = smem_u32(S.q[rc & (kQBufs - 1)]);
-                const uint32_t sfa = tmem + kSfaCol + kSfaPerStage * st;
-                const uint32_t sfb = tmem + kSfbCol + 4 * (rc & (kStages - 1));
+                const uint32_t sfa = tmem + C::kSfaCol + C::kSfaPerStage * st;
+                const uint32_t sfb = tmem + C::kSfbCol + C::kSfbPerBuf * (rc & (kStages - 1));
+                if constexpr (F8) {
+                    // K = 32 E4M3 values (32 bytes of the 128-byte row) per MMA
+                    const uint32_t a0 = smem_u32(S.a8[st]), b0 = smem_u32(S.q8[rc & (kQBufs - 1)]);
 #pragma unroll
-                for (int t = 0; t < kTilesPerStep; ++t)
+                    for (int k = 0; k < 4; ++k)
+                        mma_mxf8(tmem + b * kAccCols, smem_desc(a0 + 32 * k, 16, 1024),
+                                 smem_desc(b0 + 32 * k, 16, 1024), idesc, sfa + 4 * k, sfb + 2 * k, k > 0);
+                } else {
+                    const uint32_t a0 = smem_u32(S.a[st]), b0 = smem_u32(S.q[rc & (kQBufs - 1)]);
 #pragma unroll
-                    for (int k = 0; k < 2; ++k)
-                        mma_mxf4(tmem + b * kAccCols + 64 * t,
-                                 smem_desc(a0 + t * (kTileKeys * kKeyBytes) + 32 * k, 16, 512, 4),
-                                 smem_desc(b0 + 32 * k, 16, 512, 4), idesc, sfa + 8 * t + 4 * k,
-                                 sfb + 2 * k, k > 0);
+                    for (int t = 0; t < kTilesPerStep; ++t)
+#pragma unroll
+                        for (int k = 0; k < 2; ++k)
+                            mma_mxf4(tmem + b * kAccCols + 64 * t,
+                                     smem_desc(a0 + t * (kTileKeys * kKeyBytes) + 32 * k, 16, 512, 4),
+                                     smem_desc(b0 + 32 * k, 16, 512, 4), idesc, sfa + 8 * t + 4 * k,
+                                     sfb + 2 * k, k > 0);
+                }
                 mma_commit(&S.a_empty[st]);
                 mma_commit(&S.acc_full[b]);
                 if (++st == kStages) { st = 0; ph ^= 1u; }
@@ -243,48 +338,107 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
     } else if (warp < kEpiWarp0) {
         // ------------------------------------------------------ scale writers
-        // warp q writes TMEM lane quarter q.  Lane i handles keys 128 t + 32 c
-        // + i (tile t, column c within the tile: SFA columns 8t + c for MMA
-        // k-step 0, 8t + 4 + c for k-step 1) and heads i, 32+i (SFB columns
-        // 0..1, 2..3).
+        // warp q writes TMEM lane quarter q.  Lane i handles keys 32 c + i
+        // (SFA column group of MMA k-step s, column c) and heads i, 32 + i
+        // (two SFB columns per k-step).  The MXFP4 MMA (K = 64) takes two
+        // scales per row from bytes 0..1 of a column; the FP8 one (K = 32)
+        // one scale from byte 0.
         const int quarter = warp & 3;
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+        const int qt = threadIdx.x - 64;  // 0..127: quantiser thread (head qt / 2, dims 64 (qt & 1) ..)
         TileWalk tw(a, u0, u1);
         int64_t cur_row = -1;
         int rc = -1, st = 0;
         uint32_t ph = 0;
         bool ok = true;
-        for (int it = 0; ok && tw.next(a); ++it) {
+        // after a timed-out wait the role keeps walking its steps without
+        // waiting or touching memory, so that all 128 threads still meet at
+        // the quantiser's named barrier; ok stays uniform within each warp
+        for (int it = 0; tw.next(a); ++it) {
             const bool first_of_row = tw.row != cur_row;
             if (first_of_row) { cur_row = tw.row; ++rc; }
+            const int qb = rc & (kQBufs - 1);
+            if (QRAW && first_of_row) {
+                // quantise the row's query block straight into the MMA layout
+                if (ok && rc >= kQBufs) ok = mbar_wait(&S.q_empty[qb], uint32_t((rc / kQBufs) - 1) & 1u);
+                if (ok) {
+                    const int h = qt >> 1, half = qt & 1;
+                    const uint4* src =
+                        reinterpret_cast<const uint4*>(a.qraw + (cur_row * kHI + h) * kDI + 64 * half);
+                    uint4 v[2][4];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[i >> 2][i & 3] = src[i];
+                    uint32_t sb = 0;
+#pragma unroll
+                    for (int blk = 0; blk < 2; ++blk) {
+                        uint4 codes;
+                        sb |= quant_block32(v[blk], codes) << (8 * blk);
+                        *reinterpret_cast<uint4*>(S.q[qb] + sw64_offset(h, 2 * half + blk)) = codes;
+                    }
+                    reinterpret_cast<uint16_t*>(&S.q_sf[qb][h])[half] = uint16_t(sb);
+                    fence_proxy_async_smem();
+                }
+                ok = named_bar_and(1, 128, ok);  // every head's codes and scale bytes are written
+                if (ok && lane == 0) mbar_arrive(&S.q_full[qb]);
+            }
             // a_full of step it implies the MMA of step it - kStages is done,
             // so this stage's TMEM scale buffer is free
-            ok = mbar_wait(&S.a_full[st], ph);
-            if (!ok) break;
+            if (ok) ok = mbar_wait(&S.a_full[st], ph);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                if constexpr (F8) {
+                    float v[16];
 #pragma unroll
-            for (int t = 0; t < kTilesPerStep; ++t) {
-                uint32_t v[8];
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t wd = S.a_sf[st][32 * c + lane];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t wd = S.a_sf[st][128 * t + 32 * c + lane];
-                    v[c] = wd & 0xFFFFu;
-                    v[4 + c] = wd >> 16;
+                        for (int k = 0; k < 4; ++k) v[4 * k + c] = __uint_as_float((wd >> (8 * k)) & 0xFFu);
+                    }
+                    tmem_st16(tmem + lane_addr + C::kSfaCol + C::kSfaPerStage * st, v);
+                } else {
+#pragma unroll
+                    for (int t = 0; t < kTilesPerStep; ++t) {
+                        uint32_t v[8];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const uint32_t wd = S.a_sf[st][128 * t + 32 * c + lane];
+                            v[c] = wd & 0xFFFFu;
+                            v[4 + c] = wd >> 16;
+                        }
+                        tmem_st8(tmem + lane_addr + C::kSfaCol + C::kSfaPerStage * st + 8 * t, v);
+                    }
                 }
-                tmem_st8(tmem + lane_addr + kSfaCol + kSfaPerStage * st + 8 * t, v);
+                if (first_of_row) {
+                    uint32_t w0, w1;
+                    if (QRAW) {
+                        w0 = S.q_sf[qb][lane];
+                        w1 = S.q_sf[qb][32 + lane];
+                    } else {
+                        const uint32_t* qs = reinterpret_cast<const uint32_t*>(a.qIs) + cur_row * kHI;
+                        w0 = qs[lane];
+                        w1 = qs[32 + lane];
+                    }
+                    const uint32_t sfb = tmem + lane_addr + C::kSfbCol + C::kSfbPerBuf * (rc & (kStages - 1));
+                    if constexpr (F8) {
+                        uint32_t v[8];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            v[2 * k] = (w0 >> (8 * k)) & 0xFFu;
+                            v[2 * k + 1] = (w1 >> (8 * k)) & 0xFFu;
+                        }
+                        tmem_st8(sfb, v);
+                    } else {
+                        tmem_st4(sfb, w0 & 0xFFFFu, w1 & 0xFFFFu, w0 >> 16, w1 >> 16);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();  // the whole warp's stores are done: one arrival per warp
+                if (lane == 0) mbar_arrive(&S.sf_full[st]);
             }
-            if (first_of_row) {
-                const uint32_t* qs = reinterpret_cast<const uint32_t*>(a.qIs) + cur_row * kHI;
-                const uint32_t w0 = qs[lane], w1 = qs[32 + lane];
-                tmem_st4(tmem + lane_addr + kSfbCol + 4 * (rc & (kStages - 1)), w0 & 0xFFFFu,
-                         w1 & 0xFFFFu, w0 >> 16, w1 >> 16);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();  // the whole warp's stores are done: one arrival per warp
-            if (lane == 0) mbar_arrive(&S.sf_full[st]);
             if (++st == kStages) { st = 0; ph ^= 1u; }
         }
-    } else {
+    } else if (warp < kConvWarp0) {
         // ----------------------------------------------------------- epilogue
         const int g = (warp - kEpiWarp0) >> 2;        // group: steps with it % kEpiGroups == g
         const int sub = warp & 3;                     // TMEM lane quarter of this warp
@@ -342,6 +496,38 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 if (j < tw.ne) a.scores[cur_row * a.ld + j] = res[t];
             }
         }
+    } else if constexpr (F8) {
+        // ---------------------------------------------------------- converters
+        // E2M1 -> E4M3 (exact) of each step's keys, and of each row's query
+        // block; thread i expands row i (keys) / row i < 64 (heads).
+        const int ct = threadIdx.x - 32 * kConvWarp0;  // 0..127
+        TileWalk tw(a, u0, u1);
+        int64_t cur_row = -1;
+        int rc = -1, st = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int it = 0; ok && tw.next(a); ++it) {
+            if (tw.row != cur_row) {
+                cur_row = tw.row;
+                ++rc;
+                const int qb = rc & (kQBufs - 1);
+                // q_full of row rc implies the MMAs of row rc - kQBufs are done
+                ok = mbar_wait(&S.q_full[qb], uint32_t(rc / kQBufs) & 1u);
+                if (!ok) break;
+                if (ct < kHI) expand_row(S.q[qb], S.q8[qb], uint32_t(ct));
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.q8_full[qb]);
+            }
+            // a_full of step it implies the MMA of step it - kStages is done
+            ok = mbar_wait(&S.a_full[st], ph);
+            if (!ok) break;
+            expand_row(S.a[st], S.a8[st], uint32_t(ct));
+            fence_proxy_async_smem();
+            __syncwarp();  // one arrival per warp once all its rows are written
+            if (lane == 0) mbar_arrive(&S.a8_full[st]);
+            if (++st == kStages) { st = 0; ph ^= 1u; }
+        }
     }
     // the producer and MMA roles run on one lane: reconverge every warp so
     // that the CTA barrier (an aligned bar.sync) sees whole warps and really
@@ -368,13 +554,25 @@ static bool encode_rows64(CUtensorMap* map, const void* base, int64_t n_rows, in
                            CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
+template <bool QRAW, bool F8>
+static cudaError_t launch_variant(const CUtensorMap& map_k, const CUtensorMap& map_q, const IdxTcArgs& a,
+                                  cudaStream_t s) {
+    const size_t sm = sizeof(Smem<F8>) + 1024;
+    cudaError_t e = ensure_smem(indexer_tc_kernel<QRAW, F8>, size_t(sm));
+    if (e != cudaSuccess) return e;
+    const int grid = int(std::min<int64_t>(int64_t(Cfg<F8>::kCtasPerSm) * kNumSMs, a.units));
+    indexer_tc_kernel<QRAW, F8><<<grid, Cfg<F8>::kThreads, sm, s>>>(map_k, map_q, a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_indexer_tc(const void* qI, const void* qI_s, const float* w, const void* kI,
                               const void* kI_s, int64_t max_blocks, const int64_t* q_pos,
                               int batch, int n_q, int m, int W, float* scores, int64_t ld,
-                              cudaStream_t s) {
+                              bool q_bf16, bool fp8, cudaStream_t s) {
     IdxTcArgs a;
     a.kIs = (const uint8_t*)kI_s;
-    a.qIs = (const uint8_t*)qI_s;
+    a.qIs = q_bf16 ? nullptr : (const uint8_t*)qI_s;
+    a.qraw = q_bf16 ? (const uint16_t*)qI : nullptr;
     a.w = w; a.q_pos = q_pos; a.scores = scores; a.ld = ld; a.max_blocks = max_blocks;
     a.n_q = n_q; a.m = m; a.W = W;
     a.rows = int64_t(batch) * n_q;
@@ -382,15 +580,12 @@ cudaError_t launch_indexer_tc(const void* qI, const void* qI_s, const float* w, 
     a.units = a.rows * a.tiles_per_row;
     if (a.units == 0) return cudaSuccess;
     CUtensorMap map_k, map_q;
+    memset(&map_q, 0, sizeof(map_q));
     if (!encode_rows64(&map_k, kI, int64_t(batch) * max_blocks, kStepKeys) ||
-        !encode_rows64(&map_q, qI, a.rows * kHI, kHI))
+        (!q_bf16 && !encode_rows64(&map_q, qI, a.rows * kHI, kHI)))
         return cudaErrorInvalidValue;
-    const size_t sm = sizeof(Smem) + 1024;
-    cudaError_t e = ensure_smem(indexer_tc_kernel, size_t(sm));
-    if (e != cudaSuccess) return e;
-    const int grid = int(std::min<int64_t>(int64_t(kCtasPerSm) * kNumSMs, a.units));
-    indexer_tc_kernel<<<grid, kThreads, sm, s>>>(map_k, map_q, a);
-    return cudaGetLastError();
+    if (q_bf16) return fp8 ? launch_variant<true, true>(map_k, map_q, a, s) : launch_variant<true, false>(map_k, map_q, a, s);
+    return fp8 ? launch_variant<false, true>(map_k, map_q, a, s) : launch_variant<false, false>(map_k, map_q, a, s);
 }
 
 }  // namespace csa

@@ -23,19 +23,6 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
     return r;
 }
 
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
-    uint16_t r;
-    asm("{ .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n mov.b16 %0, {t, 0}; }"
-        : "=h"(r)
-        : "f"(hi), "f"(lo));
-    return r & 0xFFu;
-}
-
-// 2^e as a float for e in [-127, 127] (exact).
-__device__ __forceinline__ float pow2f(int e) {
-    return e >= -126 ? __int_as_float((e + 127) << 23) : __int_as_float(0x00400000);
-}
-
 template <int FMT>
 __device__ __forceinline__ float2 load_pair(const void* p, int64_t off) {
     if constexpr (FMT == CSA_F32) {

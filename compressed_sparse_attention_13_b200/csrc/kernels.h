@@ -43,7 +43,7 @@ bool indexer_tc_supported(int fmt, int HI, int dI, int64_t max_blocks, int64_t b
 cudaError_t launch_indexer_tc(const void* qI, const void* qI_s, const float* w, const void* kI,
                               const void* kI_s, int64_t max_blocks, const int64_t* q_pos,
                               int batch, int n_q, int m, int W, float* scores, int64_t ld,
-                              cudaStream_t s);
+                              bool q_bf16, bool fp8, cudaStream_t s);
 bool indexer_bf16_tc_supported(int fmt, int HI, int dI, int64_t max_blocks, int64_t batch, int n_q);
 cudaError_t launch_indexer_bf16_tc(const void* qI, const float* w, const void* kI, int64_t max_blocks,
                                    const int64_t* q_pos, int batch, int n_q, int m, int W,

@@ -332,6 +332,26 @@ __host__ __device__ constexpr uint32_t instr_desc_mxf4(uint32_t M, uint32_t N) {
     return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24);
 }
 
+// Block-scaled MMA on E4M3 operands (kind::mxf8f6f4, one E8M0 scale per 32
+// elements along K, K = 32 per instruction).  Row r of A (of B) finds its
+// scale in byte 0 of lane r % 32, column r / 32 past sfa (sfb), replicated in
+// all four lane quarters.
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// Instruction descriptor for kind::mxf8f6f4 with E8M0 scales: A and B E4M3
+// (format code 0), K-major, N >> 3 and M >> 4 (the accumulator is fp32).
+__host__ __device__ constexpr uint32_t instr_desc_mxf8_e4m3(uint32_t M, uint32_t N) {
+    return ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24);
+}
+
 // Arrive once on `bar` when every MMA issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile(
@@ -352,6 +372,19 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
 // layout a 2-D tensor copy with 64-byte swizzle writes.
 __device__ __forceinline__ uint32_t sw64_offset(uint32_t row, uint32_t chunk) {
     return row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
+}
+
+// Named barrier among `count` threads that also returns whether `pred` held
+// in every one of them.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n"
+        " selp.u32 %0, 1, 0, q;\n}"
+        : "=r"(r)
+        : "r"(uint32_t(pred)), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
 }
 
 // Named barrier among `count` threads (a multiple of 32).

@@ -103,6 +103,30 @@ typedef struct csa_params {
  *   deterministic run to run in both modes. */
 #define CSA_FLAG_BATCH_INVARIANT 0x1u
 
+/* CSA_FLAG_QI_BF16 -- the write path of the indexer queries ([WK] 基础设施:
+ *   MXFP4 on the indexer QK path; [RN] CSA: the indexer runs in FP4).  With
+ *   p->idx_fmt == CSA_MXFP4, qI is given as bf16 [..][HI][dI] and qI_scales
+ *   is not read: the indexer kernel quantises each query block to MXFP4 as it
+ *   loads it, with the rule of csa_quantize (block exponent floor(log2(max
+ *   |v|)) - 2, E2M1 codes rounded to nearest even), so the scores are those
+ *   of csa_quantize followed by the MXFP4 indexer, without the separate pass
+ *   or the stored quantised query.  Applies to indexer_score, csa_decode,
+ *   csa_decode_noalloc and csa_prefill; CSA_ERR_ARG with another idx_fmt,
+ *   CSA_ERR_UNSUPPORTED where the tensor-core indexer does not apply (HI !=
+ *   64, dI != 128, max_blocks not a multiple of 4, fewer than 128 keys). */
+#define CSA_FLAG_QI_BF16 0x2u
+
+/* CSA_FLAG_INDEXER_FP8 -- the lossless FP4 -> FP8 path ([WK] 基础设施: FP4 ->
+ *   FP8 dequantisation is lossless, so FP8 machinery is reused).  With
+ *   p->idx_fmt == CSA_MXFP4, every stored E2M1 code of the keys and queries
+ *   is expanded to the E4M3 byte of the same value (exact: E4M3 holds every
+ *   E2M1 value) and the product runs as the MXFP8 block-scaled tensor-core
+ *   MMA with the same E8M0 block scales.  Every product is the same exact
+ *   value as on the MXFP4 path; the scores may differ from it only in the
+ *   order of the fp32 additions.  Same scope and errors as CSA_FLAG_QI_BF16,
+ *   with which it combines. */
+#define CSA_FLAG_INDEXER_FP8 0x4u
+
 /* ------------------------------------------------------------------------
  * csa_compress -- softmax-gated pooling with a learned positional bias
  * ([RN] CSA: KV entries are pooled 4x along the sequence by a softmax gate
@@ -136,7 +160,8 @@ int csa_quantize(int32_t fmt, const float* src, int64_t rows, int32_t d, void* o
  *   scores[b][i][j] = sum_h w[b][i][h] * ReLU(qI[b][i][h] . kI[b][j])
  * for j < min(n_elig(q_pos[b][i]), max_blocks); other columns are not
  * written.  Accumulation in fp32.
- *   qI:        [batch][n_q][HI][dI] in p->idx_fmt (+ qI_scales)
+ *   qI:        [batch][n_q][HI][dI] in p->idx_fmt (+ qI_scales); bf16 (and
+ *              no scales) with CSA_FLAG_QI_BF16
  *   w:         float [batch][n_q][HI]
  *   kI:        [batch][max_blocks][dI] in p->idx_fmt (+ kI_scales)
  *   q_pos:     int64 [batch][n_q]

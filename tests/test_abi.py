@@ -180,3 +180,28 @@ def test_batch_invariant_plan_depends_on_the_row_only():
     ws = lambda p, b: K.csa_workspace_size(p, K.OP_SPARSE_ATTN, b, 1, 0) - 256
     assert ws(inv, 32) == 32 * ws(inv, 1)
     assert ws(dft, 1) > ws(dft, 32) / 32
+
+
+def test_indexer_write_path_flags_host_errors():
+    """CSA_FLAG_QI_BF16 / CSA_FLAG_INDEXER_FP8 belong to the MXFP4 indexer:
+    another index format is an argument error; with the bf16 query flag the
+    query scales are not needed, without it they are; shapes the tensor-core
+    indexer does not take are refused before anything is launched."""
+    lib = K.lib()
+    fake = C.c_void_p(0x1000)
+    for flags in (K.FLAG_QI_BF16, K.FLAG_INDEXER_FP8, K.FLAG_QI_BF16 | K.FLAG_INDEXER_FP8):
+        bf = K.params(4, 128, 512, 64, 512, 64, 128, 0.044, idx_fmt=K.BF16, flags=flags)
+        assert lib.indexer_score(C.byref(bf), 1, 1, fake, None, fake, fake, None, 256, fake, fake, 256,
+                                 None) == -1
+        # 32 index heads: no tensor-core MXFP4 indexer (query scales given, so only the shape fails)
+        p32 = K.params(4, 128, 512, 64, 512, 32, 128, 0.044, idx_fmt=K.MXFP4, flags=flags)
+        assert lib.indexer_score(C.byref(p32), 1, 1, fake, fake, fake, fake, fake, 256, fake, fake, 256,
+                                 None) == -3
+    # the stored-query path needs the query scales; the bf16 query path does not
+    # (it reaches the launch check of a 129-key row, not a multiple of 4)
+    mx = K.params(4, 128, 512, 64, 512, 64, 128, 0.044, idx_fmt=K.MXFP4)
+    assert lib.indexer_score(C.byref(mx), 1, 1, fake, None, fake, fake, fake, 129, fake, fake, 129,
+                             None) == -1
+    qb = K.params(4, 128, 512, 64, 512, 64, 128, 0.044, idx_fmt=K.MXFP4, flags=K.FLAG_QI_BF16)
+    assert lib.indexer_score(C.byref(qb), 1, 1, fake, None, fake, fake, fake, 129, fake, fake, 129,
+                             None) == -3
