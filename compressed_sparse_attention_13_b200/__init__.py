@@ -20,6 +20,7 @@ from dataclasses import dataclass
 
 F32, BF16, FP8_S64, MXFP4 = 0, 1, 2, 3
 OP_SPARSE_ATTN, OP_HCA_ATTN, OP_DECODE, OP_PREFILL, OP_WINDOW_ATTN = 0, 1, 2, 3, 4
+OP_SHARD_SELECT, OP_SHARD_ATTEND, OP_HCA_SHARD = 5, 6, 7
 FLAG_BATCH_INVARIANT = 0x1
 FLAG_QI_BF16 = 0x2
 FLAG_INDEXER_FP8 = 0x4
@@ -54,7 +55,8 @@ def params(m, window, top_k, n_heads, head_dim, idx_heads, idx_dim, scale,
 
 EXPORTS = ["csa_compress", "csa_quantize", "indexer_score", "topk_select", "sparse_mqa_attn",
            "hca_attn", "window_attn", "csa_decode", "csa_prefill", "csa_workspace_size",
-           "csa_device_status", "csa_strerror", "csa_version", "csa_decode_noalloc"]
+           "csa_device_status", "csa_strerror", "csa_version", "csa_decode_noalloc",
+           "csa_shard_select", "csa_shard_attend", "hca_shard_attend", "attn_merge"]
 
 
 def lib():
@@ -80,6 +82,11 @@ def lib():
                                   I64, P, P, P, P, C.c_size_t, P]
         L.csa_decode_noalloc.argtypes = [PP, I32, P, P, P, P, P, P, P, P, I64, P, I64, P, P, P,
                                          P, P, P]
+        L.csa_shard_select.argtypes = [PP, I32, P, P, P, P, P, I64, I64, P, P, P, P, C.c_size_t, P]
+        L.csa_shard_attend.argtypes = [PP, I32, P, I32, P, P, P, P, I64, I64, P, I64, P, P, P, P, P, P,
+                                       C.c_size_t, P]
+        L.hca_shard_attend.argtypes = [PP, I32, P, P, P, I64, I64, P, I64, P, P, P, P, P, C.c_size_t, P]
+        L.attn_merge.argtypes = [PP, I32, I32, P, P, P, P, P]
         L.csa_workspace_size.restype = C.c_size_t
         L.csa_workspace_size.argtypes = [PP, I32, I32, I64, I64]
         L.csa_device_status.argtypes = [P, C.POINTER(C.c_uint32), I32]
@@ -229,6 +236,37 @@ def csa_prefill(p: Params, batch: int, T: int, t0: int, raw, n_raw: int, raw_pos
         C.byref(p), batch, T, t0, _p(raw), n_raw, raw_pos0, _p(z), _p(bias), _p(q), _p(qI.data),
         _p(qI.scales), _p(w), _p(kv.data), _p(kv.scales), _p(kI.data), _p(kI.scales),
         max_blocks, _p(sinks), _p(out), _p(idx_out), wp, wb, _s(stream)))
+
+
+def csa_shard_select(p: Params, batch: int, qI: Stored, w, kI: Stored, n_entries: int, entry0: int, q_pos,
+                     cand_scores, cand_ids, workspace, stream=None):
+    wp, wb = _ws(workspace)
+    _ok("csa_shard_select", lib().csa_shard_select(
+        C.byref(p), batch, _p(qI.data), _p(qI.scales), _p(w), _p(kI.data), _p(kI.scales), n_entries, entry0,
+        _p(q_pos), _p(cand_scores), _p(cand_ids), wp, wb, _s(stream)))
+
+
+def csa_shard_attend(p: Params, batch: int, q, n_parts: int, cand_scores, cand_ids, kv: Stored,
+                     n_entries: int, entry0: int, raw, n_raw: int, raw_pos0, q_pos, part_o, part_ml,
+                     idx_out, workspace, stream=None):
+    wp, wb = _ws(workspace)
+    _ok("csa_shard_attend", lib().csa_shard_attend(
+        C.byref(p), batch, _p(q), n_parts, _p(cand_scores), _p(cand_ids), _p(kv.data), _p(kv.scales),
+        n_entries, entry0, _p(raw), n_raw, _p(raw_pos0), _p(q_pos), _p(part_o), _p(part_ml), _p(idx_out),
+        wp, wb, _s(stream)))
+
+
+def hca_shard_attend(p: Params, batch: int, q, kv: Stored, n_entries: int, entry0: int, raw, n_raw: int,
+                     raw_pos0, q_pos, part_o, part_ml, workspace, stream=None):
+    wp, wb = _ws(workspace)
+    _ok("hca_shard_attend", lib().hca_shard_attend(
+        C.byref(p), batch, _p(q), _p(kv.data), _p(kv.scales), n_entries, entry0, _p(raw), n_raw,
+        _p(raw_pos0), _p(q_pos), _p(part_o), _p(part_ml), wp, wb, _s(stream)))
+
+
+def attn_merge(p: Params, batch: int, n_parts: int, part_o, part_ml, sinks, out, stream=None):
+    _ok("attn_merge", lib().attn_merge(C.byref(p), batch, n_parts, _p(part_o), _p(part_ml), _p(sinks),
+                                       _p(out), _s(stream)))
 
 
 def csa_device_status(reset: bool = True, stream=None) -> int:

@@ -106,11 +106,15 @@ static AttnPlan plan_attn(const csa_params* p, int64_t rows, int64_t items_per_r
     return a;
 }
 
+// Attention over each row's items into `out`.  With part_ml set, the result
+// is instead the row's unnormalised partial (part_ml: max and sum per head,
+// out: fp32 O [rows][H][D]) without the sink, for a later merge with other
+// shards' partials; kv_base is the global index of kv's entry 0 (dense rows).
 static int run_attn(const csa_params* p, int batch, int n_q, const void* q, const void* kv,
                     const void* kv_s, int64_t max_entries, const int32_t* idx, const void* raw,
                     int64_t n_raw, const int64_t* raw_pos0, const int64_t* q_pos,
                     const float* sinks, void* out, void* ws, size_t ws_bytes, int64_t items_per_row,
-                    cudaStream_t s, bool pdl = false) {
+                    cudaStream_t s, bool pdl = false, float2* part_ml = nullptr, int64_t kv_base = 0) {
     const int64_t rows = int64_t(batch) * n_q;
     if (!attn_simt_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim) &&
         !attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim))
@@ -126,6 +130,12 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
     a.n_q = n_q; a.n_splits = plan.n_splits; a.out = out;
     a.part_o = (float*)ws;
     a.part_ml = (float2*)((char*)ws + plan.part_o_bytes);
+    a.partial_out = part_ml != nullptr;
+    a.kv_base = kv_base;
+    if (part_ml && plan.n_splits == 1) {  // the one split's partial is the result
+        a.part_o = (float*)out;
+        a.part_ml = part_ml;
+    }
     const bool tc = attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim) &&
                     attn_tc_rows_fit(max_entries, n_raw);
     // the CUDA-core kernel puts the query rows on the grid's y axis
@@ -138,8 +148,9 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
     if (st) return st;
     // the combine always follows this function's own attention launch
     if (plan.n_splits > 1 && !combined)
-        st = cuda_status(launch_combine(p->act_fmt, p->n_heads, p->head_dim, plan.n_splits, rows,
-                                        a.part_o, a.part_ml, sinks, out, s, /*pdl=*/true));
+        st = cuda_status(launch_combine_strided(p->act_fmt, part_ml != nullptr, p->n_heads, p->head_dim,
+                                                plan.n_splits, rows, plan.n_splits, 1, a.part_o, a.part_ml,
+                                                sinks, out, part_ml, s, /*pdl=*/true));
     return st;
 }
 
@@ -347,6 +358,18 @@ size_t csa_workspace_size(const csa_params* p, int32_t op, int32_t batch, int64_
         const size_t sel = ((size_t(rows) * p->top_k * 4) + 255) & ~size_t(255);
         return pos + scores + sel + plan_attn(p, rows, int64_t(p->top_k) + p->window).bytes() + 256;
     }
+    case CSA_OP_SHARD_SELECT: {
+        const size_t pos = ((size_t(rows) * 8) + 255) & ~size_t(255);
+        const size_t scores = ((size_t(rows) * size_t(std::max<int64_t>(n_ctx, 1)) * 4) + 255) & ~size_t(255);
+        const size_t sel = ((size_t(rows) * p->top_k * 4) + 255) & ~size_t(255);
+        return pos + scores + sel + 256;
+    }
+    case CSA_OP_SHARD_ATTEND: {
+        const size_t sel = ((size_t(rows) * p->top_k * 4) + 255) & ~size_t(255);
+        return 2 * sel + plan_attn(p, rows, int64_t(p->top_k) + p->window).bytes() + 256;
+    }
+    case CSA_OP_HCA_SHARD:
+        return plan_attn(p, rows, n_ctx + p->window).bytes() + 256;
     default:
         return 0;
     }
@@ -470,5 +493,99 @@ const char* csa_strerror(int status) {
 }
 
 const char* csa_version(void) { return "csa13 0.1.0 sm_100a"; }
+
+
+// ------------------------------------------------------------ sharded decode
+int csa_shard_select(const csa_params* p, int32_t batch, const void* qI, const void* qI_scales, const float* w,
+                     const void* kI, const void* kI_scales, int64_t n_entries, int64_t entry0,
+                     const int64_t* q_pos, float* cand_scores, int32_t* cand_ids, void* workspace,
+                     size_t ws_bytes, csa_stream_t stream) {
+    int st = check_params(p, true, false);
+    if (st) return st;
+    if (batch < 0 || n_entries < 0 || entry0 < 0 || entry0 + n_entries > INT32_MAX) return CSA_ERR_ARG;
+    if (batch == 0) return CSA_OK;
+    if (!q_pos || !cand_scores || !cand_ids || !workspace) return CSA_ERR_ARG;
+    if (ws_bytes < csa_workspace_size(p, CSA_OP_SHARD_SELECT, batch, 1, n_entries)) return CSA_ERR_WORKSPACE;
+    if (!aligned16(workspace) || !aligned16(cand_scores) || !aligned16(cand_ids)) return CSA_ERR_ALIGN;
+    const cudaStream_t s = (cudaStream_t)stream;
+    const int64_t ld = std::max<int64_t>(n_entries, 1);
+    int64_t* q_local = (int64_t*)workspace;
+    float* scores = (float*)((char*)workspace + (((size_t(batch) * 8) + 255) & ~size_t(255)));
+    int32_t* sel = (int32_t*)((char*)scores + (((size_t(batch) * ld * 4) + 255) & ~size_t(255)));
+    // the shard's eligible entries are those with entry0 + j < n_elig(t):
+    // the count n_elig seen at t - entry0 * m
+    st = cuda_status(launch_shift_positions(q_pos, q_local, batch, entry0 * int64_t(p->m), s));
+    if (st) return st;
+    if (n_entries > 0) {
+        st = indexer_score(p, batch, 1, qI, qI_scales, w, kI, kI_scales, n_entries, q_local, scores, ld, stream);
+        if (st) return st;
+    }
+    if (n_entries > 0) {
+        st = topk_impl(p, batch, 1, scores, ld, n_entries, q_local, sel, stream, false);
+        if (st) return st;
+    }
+    return cuda_status(launch_shard_candidates(batch, p->top_k, scores, ld, n_entries > 0 ? sel : nullptr, entry0,
+                                               cand_scores, cand_ids, s));
+}
+
+int csa_shard_attend(const csa_params* p, int32_t batch, const void* q, int32_t n_parts, const float* cand_scores,
+                     const int32_t* cand_ids, const void* kv, const void* kv_scales, int64_t n_entries,
+                     int64_t entry0, const void* raw, int64_t n_raw, const int64_t* raw_pos0,
+                     const int64_t* q_pos, float* part_o, float* part_ml, int32_t* idx_out, void* workspace,
+                     size_t ws_bytes, csa_stream_t stream) {
+    int st = check_params(p, false, true);
+    if (st) return st;
+    if (p->top_k <= 0 || batch < 0 || n_parts <= 0 || n_entries < 0 || entry0 < 0) return CSA_ERR_ARG;
+    if (batch == 0) return CSA_OK;
+    if (!topk_merge_supported(n_parts * p->top_k) || p->top_k > 4096) return CSA_ERR_UNSUPPORTED;
+    if (!cand_scores || !cand_ids || !part_ml || !workspace) return CSA_ERR_ARG;
+    st = check_attn_ptrs(q, kv, kv_scales, p->kv_fmt, raw, n_raw, raw_pos0, q_pos, part_o, n_entries > 0);
+    if (st) return st;
+    if (!aligned16(part_ml) || !aligned16(workspace)) return CSA_ERR_ALIGN;
+    if (ws_bytes < csa_workspace_size(p, CSA_OP_SHARD_ATTEND, batch, 1, n_entries)) return CSA_ERR_WORKSPACE;
+    const cudaStream_t s = (cudaStream_t)stream;
+    const size_t sel_bytes = ((size_t(batch) * p->top_k * 4) + 255) & ~size_t(255);
+    int32_t* sel_global = idx_out ? idx_out : (int32_t*)workspace;
+    int32_t* sel_local = (int32_t*)((char*)workspace + sel_bytes);
+    st = cuda_status(launch_topk_merge(batch, n_parts, p->top_k, cand_scores, cand_ids, entry0, n_entries,
+                                       sel_global, sel_local, s));
+    if (st) return st;
+    return run_attn(p, batch, 1, q, kv, kv_scales, n_entries, sel_local, raw, n_raw, raw_pos0, q_pos, nullptr,
+                    part_o, (char*)workspace + 2 * sel_bytes, ws_bytes - 2 * sel_bytes,
+                    int64_t(p->top_k) + p->window, s, false, (float2*)part_ml);
+}
+
+int hca_shard_attend(const csa_params* p, int32_t batch, const void* q, const void* kv, const void* kv_scales,
+                     int64_t n_entries, int64_t entry0, const void* raw, int64_t n_raw,
+                     const int64_t* raw_pos0, const int64_t* q_pos, float* part_o, float* part_ml,
+                     void* workspace, size_t ws_bytes, csa_stream_t stream) {
+    int st = check_params(p, false, true);
+    if (st) return st;
+    if (batch < 0 || n_entries < 0 || entry0 < 0) return CSA_ERR_ARG;
+    if (batch == 0) return CSA_OK;
+    if (!part_ml) return CSA_ERR_ARG;
+    st = check_attn_ptrs(q, kv, kv_scales, p->kv_fmt, raw, n_raw, raw_pos0, q_pos, part_o, n_entries > 0);
+    if (st) return st;
+    if (!aligned16(part_ml)) return CSA_ERR_ALIGN;
+    if (ws_bytes < csa_workspace_size(p, CSA_OP_HCA_SHARD, batch, 1, n_entries)) return CSA_ERR_WORKSPACE;
+    return run_attn(p, batch, 1, q, kv, kv_scales, n_entries, nullptr, raw, n_raw, raw_pos0, q_pos, nullptr,
+                    part_o, workspace, ws_bytes, n_entries + p->window, (cudaStream_t)stream, false,
+                    (float2*)part_ml, entry0);
+}
+
+int attn_merge(const csa_params* p, int32_t batch, int32_t n_parts, const float* part_o, const float* part_ml,
+               const float* sinks, void* out, csa_stream_t stream) {
+    int st = check_params(p, false, true);
+    if (st) return st;
+    if (batch < 0 || n_parts <= 0) return CSA_ERR_ARG;
+    if (n_parts > 64) return CSA_ERR_UNSUPPORTED;
+    if (batch == 0) return CSA_OK;
+    if (!part_o || !part_ml || !out) return CSA_ERR_ARG;
+    if (!aligned16(part_o) || !aligned16(part_ml) || !aligned16(out)) return CSA_ERR_ALIGN;
+    if ((p->head_dim % 4) != 0) return CSA_ERR_UNSUPPORTED;
+    return cuda_status(launch_combine_strided(p->act_fmt, false, p->n_heads, p->head_dim, n_parts, batch, 1, batch,
+                                              part_o, (const float2*)part_ml, sinks, out, nullptr,
+                                              (cudaStream_t)stream));
+}
 
 }  // extern "C"

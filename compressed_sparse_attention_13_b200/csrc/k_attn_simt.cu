@@ -32,7 +32,7 @@ __device__ __forceinline__ RowSlots row_slots(const AttnArgs& a, int64_t row) {
     RowSlots r;
     const int64_t b = row / a.n_q;
     const int64_t t = a.q_pos[row];
-    r.n_kv = a.idx ? a.k : min(n_elig(t, a.m, a.W), a.max_entries);
+    r.n_kv = a.idx ? a.k : min(max(n_elig(t, a.m, a.W) - a.kv_base, int64_t(0)), a.max_entries);
     const int64_t p0 = a.raw_pos0[b];
     const int64_t lo = max(max(t - a.W + 1, int64_t(0)), p0);
     const int64_t hi = min(t + 1, p0 + a.n_raw);
@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_simt_kernel(AttnArgs a) 
     }
     __syncthreads();
     const float m_run = m_s[my_h], l_run = l_s[my_h];
-    if (a.n_splits == 1) {
+    if (a.n_splits == 1 && !a.partial_out) {
         float den = l_run, f = 1.f;
         if (a.sinks) {
             const float sg = a.sinks[my_h];
@@ -185,43 +185,57 @@ static cudaError_t launch_attn_t(const AttnArgs& a, int64_t rows, cudaStream_t s
     return cudaGetLastError();
 }
 
-// Combine split partials: o = sum_s e^(m_s-M) O_s / (sum_s e^(m_s-M) l_s + e^(sink-M)).
-// One CTA per (row, head), 128 threads x 4 dims (D = 512; other widths loop).
-// The per-split weights are computed once into shared memory, then each
-// thread accumulates float4 slices with the split loads issued four at a time.
-template <int ACT>
-__global__ void __launch_bounds__(128) combine_kernel(int H, int D, int n_splits,
-                                                      const float* __restrict__ part_o,
+// Split-K LSE combine of a row's partial attention results ([RN] CSA / HCA:
+// one softmax over all attended items and the sink).  Partial s of row r is
+// item r * row_stride + s * split_stride of part_o ([item][H][D] fp32, the
+// unnormalised sum relative to the item's running max) and part_ml ([item][H]:
+// max in natural-log units, sum of exponentials).  The per-split weights are
+// computed once into shared memory, then each thread accumulates float4
+// slices with the split loads issued four at a time.
+//   PARTIAL = false: out = sum_s w_s O_s / (sum_s w_s l_s + e^(sink - M)) in
+//     the activation format (the sink, if any, takes part in the max M).
+//   PARTIAL = true: the merged partial itself, with no sink: out (fp32) =
+//     sum_s w_s O_s and out_ml = (M, sum_s w_s l_s), M the max over splits.
+template <int ACT, bool PARTIAL>
+__global__ void __launch_bounds__(128) combine_kernel(int H, int D, int n_splits, int64_t row_stride,
+                                                      int64_t split_stride, const float* __restrict__ part_o,
                                                       const float2* __restrict__ part_ml,
-                                                      const float* __restrict__ sinks, void* out) {
+                                                      const float* __restrict__ sinks, void* out,
+                                                      float2* out_ml) {
     __shared__ float wgt[64];
     __shared__ float inv_s;
     pdl_wait();  // the partials come from the attention kernel before it
     const int64_t row = blockIdx.x;
     const int h = blockIdx.y;
-    const float2* ml = part_ml + row * n_splits * H + h;
+    const float* sk = PARTIAL ? nullptr : sinks;
+    auto ml_of = [&](int s) { return part_ml[(row * row_stride + s * split_stride) * H + h]; };
     if (threadIdx.x < 32) {
-        float M = sinks ? sinks[h] : -INFINITY;
-        for (int s = threadIdx.x; s < n_splits; s += 32) M = fmaxf(M, ml[s * H].x);
+        float M = sk ? sk[h] : -INFINITY;
+        for (int s = threadIdx.x; s < n_splits; s += 32) M = fmaxf(M, ml_of(s).x);
         M = warp_max(M);
         float den = 0.f;
         for (int s = threadIdx.x; s < n_splits; s += 32) {
-            const float2 v = ml[s * H];
+            const float2 v = ml_of(s);
             const float w = v.x == -INFINITY ? 0.f : expf(v.x - M);
             wgt[s] = w;
             den += w * v.y;
         }
         den = warp_sum(den);
         if (threadIdx.x == 0) {
-            if (sinks && M != -INFINITY) den += expf(sinks[h] - M);
-            inv_s = den > 0.f ? 1.f / den : 0.f;
+            if (sk && M != -INFINITY) den += expf(sk[h] - M);
+            if (PARTIAL) {
+                out_ml[row * H + h] = make_float2(M, den);
+                inv_s = 1.f;
+            } else {
+                inv_s = den > 0.f ? 1.f / den : 0.f;
+            }
         }
     }
     __syncthreads();
     const float inv = inv_s;
-    const int64_t stride = int64_t(H) * D;  // between splits
+    const int64_t stride = split_stride * H * D;  // between splits
     for (int c = 4 * threadIdx.x; c < D; c += 4 * blockDim.x) {
-        const float* base = part_o + (row * n_splits * H + h) * int64_t(D) + c;
+        const float* base = part_o + (row * row_stride * H + h) * int64_t(D) + c;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         int s = 0;
         for (; s + 4 <= n_splits; s += 4) {
@@ -244,7 +258,7 @@ __global__ void __launch_bounds__(128) combine_kernel(int H, int D, int n_splits
             acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
         }
         const int64_t o = (row * H + h) * int64_t(D) + c;
-        if constexpr (ACT == CSA_F32) {
+        if constexpr (PARTIAL || ACT == CSA_F32) {
             *reinterpret_cast<float4*>((float*)out + o) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
         } else {
             __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
@@ -257,18 +271,28 @@ __global__ void __launch_bounds__(128) combine_kernel(int H, int D, int n_splits
     }
 }
 
+cudaError_t launch_combine_strided(int act, bool partial, int H, int D, int n_splits, int64_t rows,
+                                   int64_t row_stride, int64_t split_stride, const float* part_o,
+                                   const float2* part_ml, const float* sinks, void* out, float2* out_ml,
+                                   cudaStream_t s, bool pdl) {
+    if (rows == 0) return cudaSuccess;
+    if (n_splits > 64) return cudaErrorInvalidValue;  // the weights live in a 64-entry table
+    const dim3 grid{unsigned(rows), unsigned(H)};
+    if (partial)
+        return launch_ex(combine_kernel<CSA_F32, true>, grid, dim3(128), 0, s, pdl, H, D, n_splits, row_stride,
+                         split_stride, part_o, part_ml, sinks, out, out_ml);
+    if (act == CSA_F32)
+        return launch_ex(combine_kernel<CSA_F32, false>, grid, dim3(128), 0, s, pdl, H, D, n_splits, row_stride,
+                         split_stride, part_o, part_ml, sinks, out, out_ml);
+    return launch_ex(combine_kernel<CSA_BF16, false>, grid, dim3(128), 0, s, pdl, H, D, n_splits, row_stride,
+                     split_stride, part_o, part_ml, sinks, out, out_ml);
+}
+
 cudaError_t launch_combine(int act, int H, int D, int n_splits, int64_t rows, const float* part_o,
                            const float2* part_ml, const float* sinks, void* out, cudaStream_t s,
                            bool pdl) {
-    if (rows == 0) return cudaSuccess;
-    const dim3 grid{unsigned(rows), unsigned(H)};
-    if (act == CSA_F32)
-        return launch_ex(combine_kernel<CSA_F32>, grid, dim3(128), 0, s, pdl, H, D, n_splits, part_o,
-                         part_ml, sinks, out);
-    else
-        return launch_ex(combine_kernel<CSA_BF16>, grid, dim3(128), 0, s, pdl, H, D, n_splits, part_o,
-                         part_ml, sinks, out);
-    return cudaGetLastError();
+    return launch_combine_strided(act, false, H, D, n_splits, rows, n_splits, 1, part_o, part_ml, sinks, out,
+                                  nullptr, s, pdl);
 }
 
 // Dispatch on (dims per thread, activation format, entry format).

@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int split = blockIdx.x;
     const int64_t b = row / a.n_q;
     const int64_t t = a.q_pos[row];
-    const int64_t n_kv = a.idx ? a.k : min(n_elig(t, a.m, a.W), a.max_entries);
+    const int64_t n_kv = a.idx ? a.k : min(max(n_elig(t, a.m, a.W) - a.kv_base, int64_t(0)), a.max_entries);
     const int64_t p0 = a.raw_pos0[b];
     const int64_t win_lo = max(max(t - a.W + 1, int64_t(0)), p0);
     const int64_t n_win = max(int64_t(0), min(t + 1, p0 + a.n_raw) - win_lo);
@@ -549,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // ----------------------------------------------------------- epilogue
         if (head_lane) {
-            if (a.n_splits == 1) {
+            if (a.n_splits == 1 && !a.partial_out) {
                 float f = 1.f, den = l_run;
                 if (a.sinks) {
                     const float sg = a.sinks[h] * kLog2e;
@@ -578,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // O goes there as [64 heads][512 dims] (fp32 partials, or the final
         // bf16 output) and leaves in a few bulk stores.
         const int e = sub * 32 + lane;
-        const bool final_out = a.n_splits == 1;
+        const bool final_out = a.n_splits == 1 && !a.partial_out;
         float* so32 = reinterpret_cast<float*>(&S.kv[0][0][0]);
         __nv_bfloat16* so16 = reinterpret_cast<__nv_bfloat16*>(&S.kv[0][0][0]);
         for (int qt = 0; qt < 4; ++qt) {
@@ -759,7 +759,7 @@ static cudaError_t launch_attn_tc_fmt(AttnArgs a, int64_t rows, cudaStream_t s, 
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     // The splits of a row combine inside the kernel when they fit one portable
     // cluster and such clusters can be scheduled; otherwise launch_combine runs.
-    if (a.n_splits >= 2 && a.n_splits <= 8) {
+    if (a.n_splits >= 2 && a.n_splits <= 8 && !a.partial_out) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         if (cluster_fits<KVF>(cfg)) {

@@ -27,6 +27,9 @@ struct AttnArgs {
     int fused_combine;        // tensor-core kernel: the splits of a row form a cluster and
                               // combine through distributed shared memory (set by the launcher)
     int64_t row_base;         // tensor-core kernel: first row of this launch (set by the launcher)
+    int partial_out;          // write (m, l, O) partials even with one split; no sink applied
+    int64_t kv_base;          // global index of entry 0 of kv (a shard); dense rows attend to
+                              // entries j with kv_base + j < n_elig(t)
 };
 
 cudaError_t launch_compress(int in_fmt, int out_fmt, const void* x, const void* z,
@@ -66,5 +69,30 @@ bool attn_simt_supported(int act, int kvf, int H, int D);
 cudaError_t launch_combine(int act, int H, int D, int n_splits, int64_t rows, const float* part_o,
                            const float2* part_ml, const float* sinks, void* out, cudaStream_t s,
                            bool pdl = false);
+// The same with explicit strides (partial s of row r is item r * row_stride +
+// s * split_stride); partial = true writes the merged (M, L) and fp32 O
+// without a sink instead of the normalised output.
+cudaError_t launch_combine_strided(int act, bool partial, int H, int D, int n_splits, int64_t rows,
+                                   int64_t row_stride, int64_t split_stride, const float* part_o,
+                                   const float2* part_ml, const float* sinks, void* out, float2* out_ml,
+                                   cudaStream_t s, bool pdl = false);
+
+// Sharded decode helpers (k_shard.cu).
+// q_local[i] = q_pos[i] - delta: a shard whose first entry is entry0 sees the
+// eligible count n_elig(t) - entry0 at position t - entry0 * m.
+cudaError_t launch_shift_positions(const int64_t* q_pos, int64_t* q_local, int64_t n, int64_t delta,
+                                   cudaStream_t s);
+// The shard's local top-k as candidates: (score, entry0 + local id), or
+// (-inf, -1) for an empty slot.
+cudaError_t launch_shard_candidates(int64_t rows, int k, const float* scores, int64_t ld, const int32_t* sel,
+                                    int64_t entry0, float* cand_scores, int32_t* cand_ids, cudaStream_t s);
+// Global top-k of each row's candidates (gathered rank-major: [n_parts][rows][k]),
+// ranked by score and then by the smaller id; writes the selection as
+// ascending global ids (-1 padded) and the part in [entry0, entry0 + n_entries)
+// as ascending local ids (-1 padded).
+bool topk_merge_supported(int n_cand);
+cudaError_t launch_topk_merge(int64_t rows, int n_parts, int k, const float* cand_scores, const int32_t* cand_ids,
+                              int64_t entry0, int64_t n_entries, int32_t* sel_global, int32_t* sel_local,
+                              cudaStream_t s);
 
 }  // namespace csa

@@ -283,6 +283,9 @@ int csa_prefill(const csa_params* p, int32_t batch, int64_t T, int64_t t0, const
 #define CSA_OP_DECODE 2
 #define CSA_OP_PREFILL 3
 #define CSA_OP_WINDOW_ATTN 4
+#define CSA_OP_SHARD_SELECT 5
+#define CSA_OP_SHARD_ATTEND 6
+#define CSA_OP_HCA_SHARD 7
 
 /* Bytes of workspace an operation needs (0 on bad arguments; SIZE_MAX when
  * the size does not fit in size_t, which no buffer satisfies).  n_ctx is
@@ -337,6 +340,75 @@ int csa_decode_noalloc(const csa_params* p, int32_t batch, const void* q, const 
                        int64_t max_blocks, const void* raw, int64_t n_raw,
                        const int64_t* raw_pos0, const int64_t* q_pos, const float* sinks,
                        void* out, int32_t* idx_out, csa_stream_t stream);
+
+/* ========================================================================
+ * Sharded decode: one sequence's pooled entries split over ranks along the
+ * entry axis, for contexts of 1M tokens and beyond ([RN] 架構實現 and the
+ * paper summary: 1M-token context; a CSA layer takes the top-k of all
+ * visible entries, an HCA layer attends to all of them).  Rank r holds the
+ * contiguous entries [entry0, entry0 + n_entries) of every sequence of the
+ * batch (local entry j is global entry entry0 + j); exactly one rank passes
+ * the raw window (n_raw > 0), the others n_raw = 0.  Per CSA layer:
+ *   1. csa_shard_select on every rank -> k candidates (score, global id);
+ *   2. all-gather of the candidates, rank-major: [n_parts][batch][k];
+ *   3. csa_shard_attend on every rank -> the exact global top-k (the union
+ *      of the shards' top-k under the order score descending, id ascending
+ *      contains it), attention over the selected entries this rank holds
+ *      (and the window) as an unnormalised partial;
+ *   4. all-gather of the partials, rank-major; attn_merge -> the output.
+ * Per HCA layer: hca_shard_attend, all-gather, attn_merge.  The partial of
+ * a row is O [H][D] fp32 (sum of e^(logit - M) v over this rank's items)
+ * and (M, L) per head (float pairs: M in natural-log units, L the sum of
+ * e^(logit - M)); a rank with no item gives M = -inf, L = 0, O = 0.  The
+ * exchange itself is the caller's (an NCCL all-gather); these calls only
+ * read and write device memory on `stream`.
+ * ======================================================================== */
+
+/* csa_shard_select -- the indexer over this rank's keys and their local
+ * top-k.  Key j is scored for query t only if entry0 + j < n_elig(t).
+ *   qI, qI_scales, w, q_pos as for csa_decode (p->flags apply); kI: this
+ *   rank's keys [batch][n_entries][dI] in p->idx_fmt.
+ *   cand_scores float [batch][k], cand_ids int32 [batch][k]: the local top-k
+ *   (ids global, in ascending order), padded with (-inf, -1).
+ *   workspace: >= csa_workspace_size(p, CSA_OP_SHARD_SELECT, batch, 1, n_entries) */
+int csa_shard_select(const csa_params* p, int32_t batch, const void* qI, const void* qI_scales, const float* w,
+                     const void* kI, const void* kI_scales, int64_t n_entries, int64_t entry0,
+                     const int64_t* q_pos, float* cand_scores, int32_t* cand_ids, void* workspace,
+                     size_t ws_bytes, csa_stream_t stream);
+
+/* csa_shard_attend -- the global top-k of the gathered candidates and this
+ * rank's partial of the sparse attention.
+ *   cand_scores, cand_ids: [n_parts][batch][k] (every rank's csa_shard_select
+ *   output, rank-major); n_parts * k <= 16384 and k <= 4096, else
+ *   CSA_ERR_UNSUPPORTED.  kv: this rank's entries [batch][n_entries][d] in
+ *   p->kv_fmt; raw / n_raw / raw_pos0: the window as for csa_decode on the
+ *   rank that attends to it, n_raw = 0 (raw may be NULL) elsewhere.
+ *   part_o float [batch][H][d], part_ml float [batch][H][2]: the partial.
+ *   idx_out int32 [batch][k] (may be NULL): the global selection, ascending
+ *   ids, -1 padded -- the same on every rank.
+ *   workspace: >= csa_workspace_size(p, CSA_OP_SHARD_ATTEND, batch, 1, n_entries) */
+int csa_shard_attend(const csa_params* p, int32_t batch, const void* q, int32_t n_parts, const float* cand_scores,
+                     const int32_t* cand_ids, const void* kv, const void* kv_scales, int64_t n_entries,
+                     int64_t entry0, const void* raw, int64_t n_raw, const int64_t* raw_pos0,
+                     const int64_t* q_pos, float* part_o, float* part_ml, int32_t* idx_out, void* workspace,
+                     size_t ws_bytes, csa_stream_t stream);
+
+/* hca_shard_attend -- this rank's partial of the dense HCA attention: local
+ * entries j with entry0 + j < n_elig(t), plus the window on the rank that
+ * passes it.  Arguments as csa_shard_attend without the candidates.
+ *   workspace: >= csa_workspace_size(p, CSA_OP_HCA_SHARD, batch, 1, n_entries) */
+int hca_shard_attend(const csa_params* p, int32_t batch, const void* q, const void* kv, const void* kv_scales,
+                     int64_t n_entries, int64_t entry0, const void* raw, int64_t n_raw,
+                     const int64_t* raw_pos0, const int64_t* q_pos, float* part_o, float* part_ml,
+                     void* workspace, size_t ws_bytes, csa_stream_t stream);
+
+/* attn_merge -- LSE merge of n_parts partials per row (rank-major:
+ * part_o [n_parts][batch][H][d], part_ml [n_parts][batch][H][2]) with the
+ * per-head sink (NULL: none):
+ *   out = sum_r e^(M_r - M) O_r / (sum_r e^(M_r - M) L_r + e^(sink - M))
+ * in p->act_fmt [batch][H][d].  n_parts <= 64 (else CSA_ERR_UNSUPPORTED). */
+int attn_merge(const csa_params* p, int32_t batch, int32_t n_parts, const float* part_o, const float* part_ml,
+               const float* sinks, void* out, csa_stream_t stream);
 
 /* Synchronise `stream`, return the device status word (CSA_DEV_* bits) in
  * *flags, and clear it if `reset` is non-zero.  The word is shared by every

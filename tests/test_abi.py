@@ -205,3 +205,31 @@ def test_indexer_write_path_flags_host_errors():
     qb = K.params(4, 128, 512, 64, 512, 64, 128, 0.044, idx_fmt=K.MXFP4, flags=K.FLAG_QI_BF16)
     assert lib.indexer_score(C.byref(qb), 1, 1, fake, None, fake, fake, fake, 129, fake, fake, 129,
                              None) == -3
+
+
+def test_sharded_decode_host_errors():
+    """Argument checks of the sharded entry points, before any launch."""
+    lib = K.lib()
+    p = K.params(4, 128, 512, 64, 512, 64, 128, 0.044)
+    P = C.byref(p)
+    fake = C.c_void_p(0x1000)
+    # select: negative entry offset; a workspace below the plan
+    assert lib.csa_shard_select(P, 1, fake, fake, fake, fake, fake, 1024, -1, fake, fake, fake, fake,
+                                1 << 20, None) == -1
+    need = lib.csa_workspace_size(P, K.OP_SHARD_SELECT, 2, 1, 4096)
+    assert need >= 2 * 4096 * 4 + 2 * 512 * 4
+    assert lib.csa_shard_select(P, 2, fake, fake, fake, fake, fake, 4096, 0, fake, fake, fake, fake,
+                                need - 1, None) == -4
+    # attend: no parts; too many candidates for the merge; no partial output
+    args = lambda n_parts, pml: (P, 1, fake, n_parts, fake, fake, fake, fake, 1024, 0, None, 0, fake, fake,
+                                 fake, pml, None, fake, 1 << 30, None)
+    assert lib.csa_shard_attend(*args(0, fake)) == -1
+    assert lib.csa_shard_attend(*args(33, fake)) == -3      # 33 x 512 > 16384 candidates
+    assert lib.csa_shard_attend(*args(4, None)) == -1
+    # HCA partial without its (M, L) output; merge over no or too many parts
+    assert lib.hca_shard_attend(P, 1, fake, fake, fake, 1024, 0, None, 0, fake, fake, fake, None, fake,
+                                1 << 30, None) == -1
+    assert lib.attn_merge(P, 1, 0, fake, fake, None, fake, None) == -1
+    assert lib.attn_merge(P, 1, 65, fake, fake, None, fake, None) == -3
+    odd = C.c_void_p(0x1004)
+    assert lib.attn_merge(P, 1, 2, odd, fake, None, fake, None) == -2
