@@ -23,6 +23,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -355,7 +356,8 @@ def run_ours(args):
                 "prefill": lambda: bench_prefill(dev, flush, stream, bf16_peak),
                 "stack": lambda: bench_stack(dev, flush, stream, hbm_peak, bf16_peak),
                 "schedule": lambda: bench_schedule(dev, flush, stream, hbm_peak),
-                "indexer": lambda: bench_indexer_variants(args, dev, flush, stream, hbm_peak)}
+                "indexer": lambda: bench_indexer_variants(args, dev, flush, stream, hbm_peak),
+                "shard": lambda: bench_shard(args, dev, flush, stream)}
         print(json.dumps({n: legs[n]() for n in args.only_legs.split(",")}), flush=True)
         return
 
@@ -468,7 +470,7 @@ def run_ours(args):
         "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
     }
-    legs = set(args.legs.split(",")) if args.legs else {"hca", "indexer", "prefill", "stack", "schedule"}
+    legs = set(args.legs.split(",")) if args.legs else {"hca", "indexer", "shard", "prefill", "stack", "schedule"}
     if world == 1 and rank == 0 and not args.no_extra:
         if "hca" in legs:
             result["hca_decode"] = bench_hca(args, dev, flush, stream, hbm_peak)
@@ -480,7 +482,8 @@ def run_ours(args):
             except Exception as exc:  # an extra leg must not lose the main line
                 result["indexer_write_path"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
         torch.cuda.empty_cache()
-        for key, name, leg in (("prefill_8k_bf16", "prefill", lambda: bench_prefill(dev, flush, stream, bf16_peak)),
+        for key, name, leg in (("sharded_decode_1m", "shard", lambda: bench_shard(args, dev, flush, stream)),
+                               ("prefill_8k_bf16", "prefill", lambda: bench_prefill(dev, flush, stream, bf16_peak)),
                                ("stack_c4", "stack", lambda: bench_stack(dev, flush, stream, hbm_peak, bf16_peak)),
                                ("schedule_v4_pro", "schedule", lambda: bench_schedule(dev, flush, stream, hbm_peak))):
             if name not in legs:
@@ -584,6 +587,74 @@ def bench_indexer_variants(args, dev, flush, stream, hbm_peak):
         t = statistics.mean(time_steps(graphed(fn), args.steps, args.warmup, flush, stream))
         res[name] = {"us": round(t * 1e3, 2), "key_gbs": round(key_bytes / (t / 1e3) / 1e9, 1),
                      "frac": round(key_bytes / (t / 1e3) / 1e9 / hbm_peak, 4)}
+    assert K.csa_device_status(reset=True) == 0
+    return res
+
+
+def bench_shard(args, dev, flush, stream, world=8):
+    """One 1M-token sequence (batch 1) split over `world` ranks, emulated on
+    this GPU: every rank's phases are timed one by one (graph-replayed after
+    an L2 flush), the per-GPU step is the slowest rank's select + attend plus
+    the merge; the exchanges (two all-gathers of a few KB to a few MB) are not
+    timed here (one GPU).  The unsharded call on the whole cache is timed
+    beside it."""
+    import torch
+
+    import compressed_sparse_attention_13_b200 as K
+    from compressed_sparse_attention_13_b200 import shard as SH
+    from synth import tensor_torch
+
+    N, H, d, HI, dI, W, k = 1 << 20, 64, 512, 64, 128, 128, 1024
+    res = {"workload": f"one sequence at 1M tokens sharded over {world} emulated ranks", "ranks": world}
+    t_of = lambda fn: statistics.mean(time_steps(graphed(fn), args.steps, args.warmup, flush, stream)) * 1e3
+
+    def st(name, rows, width, fmt):
+        v = tensor_torch(0, f"shard/{name}", (rows, width), device=dev)
+        o = K.empty_stored(fmt, rows, width, device=dev)
+        K.csa_quantize(v, o)
+        return o
+
+    q = tensor_torch(0, "shard/q", (1, H, d), dtype="bf16", device=dev)
+    win = tensor_torch(0, "shard/win", (1, W, d), dtype="bf16", device=dev)
+    sinks = tensor_torch(0, "shard/sinks", (H,), device=dev)
+    q_pos = torch.full((1,), N, dtype=torch.int64, device=dev)
+    raw_pos0 = q_pos - W + 1
+    out = torch.empty(1, H, d, dtype=torch.bfloat16, device=dev)
+    for kind, m in (("csa", 4), ("hca", 128)):
+        nb = N // m
+        p = K.params(m, W, k if kind == "csa" else 1, H, d, HI, dI, 1 / math.sqrt(d), K.BF16, K.FP8_S64, K.MXFP4)
+        kv = st(f"{kind}/kv", nb, d, K.FP8_S64)
+        kI = st("csa/kI", nb, dI, K.MXFP4) if kind == "csa" else None
+        shards = SH.make_shards(kv, kI, 1, nb, world)
+        r = {"entries": nb}
+        if kind == "csa":
+            qI = st("csa/qI", HI, dI, K.MXFP4)
+            wt = tensor_torch(0, "shard/w", (1, HI), 0.1, device=dev)
+            cand = [SH.csa_select(p, 1, qI, wt, sh, q_pos, dev) for sh in shards]
+            all_s, all_i = torch.stack([c[0] for c in cand]), torch.stack([c[1] for c in cand])
+            r["select_us"] = [round(t_of(lambda sh=sh: SH.csa_select(p, 1, qI, wt, sh, q_pos, dev)), 2)
+                              for sh in shards]
+            r["attend_us"] = [round(t_of(lambda sh=sh: SH.csa_attend(p, 1, q, all_s, all_i, sh, win, W, raw_pos0,
+                                                                     q_pos, None, dev)), 2) for sh in shards]
+            parts = [SH.csa_attend(p, 1, q, all_s, all_i, sh, win, W, raw_pos0, q_pos, None, dev) for sh in shards]
+            ws = torch.empty(K.csa_workspace_size(p, K.OP_DECODE, 1, 1, nb), dtype=torch.uint8, device=dev)
+            sel = torch.empty(1, k, dtype=torch.int32, device=dev)
+            r["unsharded_us"] = round(t_of(lambda: K.csa_decode(p, 1, q, qI, wt, kv, kI, nb, win, W, raw_pos0,
+                                                                q_pos, sinks, out, sel, ws)), 2)
+        else:
+            r["attend_us"] = [round(t_of(lambda sh=sh: SH.hca_attend(p, 1, q, sh, win, W, raw_pos0, q_pos, dev)), 2)
+                              for sh in shards]
+            parts = [SH.hca_attend(p, 1, q, sh, win, W, raw_pos0, q_pos, dev) for sh in shards]
+            ws = torch.empty(K.csa_workspace_size(p, K.OP_HCA_ATTN, 1, 1, nb), dtype=torch.uint8, device=dev)
+            r["unsharded_us"] = round(t_of(lambda: K.hca_attn(p, 1, 1, q, kv, nb, win, W, raw_pos0, q_pos, sinks,
+                                                              out, ws)), 2)
+        all_o, all_ml = torch.stack([x[0] for x in parts]), torch.stack([x[1] for x in parts])
+        r["merge_us"] = round(t_of(lambda: SH.merge(p, 1, all_o, all_ml, sinks, out)), 2)
+        r["per_gpu_compute_us"] = round(max(r.get("select_us", [0.0])) + max(r["attend_us"]) + r["merge_us"], 2)
+        r["exchange_bytes_per_rank"] = SH.exchange_bytes(1, k, H, d, csa=kind == "csa")
+        res[kind] = r
+        del kv, kI, shards, parts, all_o, all_ml
+        torch.cuda.empty_cache()
     assert K.csa_device_status(reset=True) == 0
     return res
 
@@ -1048,10 +1119,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true", help="skip the extra legs")
-    ap.add_argument("--legs", default="", help="extra legs to run, comma-separated among hca, indexer, prefill, "
-                    "stack, schedule (default: all)")
+    ap.add_argument("--legs", default="", help="extra legs to run, comma-separated among hca, indexer, shard, "
+                    "prefill, stack, schedule (default: all)")
     ap.add_argument("--only-legs", default="", help="run only these extra legs (comma-separated among "
-                    "hca, indexer, prefill, stack, schedule) and print their results, without the main line")
+                    "hca, indexer, shard, prefill, stack, schedule) and print their results, without the main line")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--case", default="", help="run one small named workload (decode_128k_b32, hca_1m_b8, "

@@ -366,7 +366,8 @@ size_t csa_workspace_size(const csa_params* p, int32_t op, int32_t batch, int64_
     }
     case CSA_OP_SHARD_ATTEND: {
         const size_t sel = ((size_t(rows) * p->top_k * 4) + 255) & ~size_t(255);
-        return 2 * sel + plan_attn(p, rows, int64_t(p->top_k) + p->window).bytes() + 256;
+        const size_t merge = topk_merge_workspace(rows, p->top_k);
+        return 2 * sel + std::max(merge, plan_attn(p, rows, int64_t(p->top_k) + p->window).bytes()) + 256;
     }
     case CSA_OP_HCA_SHARD:
         return plan_attn(p, rows, n_ctx + p->window).bytes() + 256;
@@ -537,7 +538,7 @@ int csa_shard_attend(const csa_params* p, int32_t batch, const void* q, int32_t 
     if (st) return st;
     if (p->top_k <= 0 || batch < 0 || n_parts <= 0 || n_entries < 0 || entry0 < 0) return CSA_ERR_ARG;
     if (batch == 0) return CSA_OK;
-    if (!topk_merge_supported(n_parts * p->top_k) || p->top_k > 4096) return CSA_ERR_UNSUPPORTED;
+    if (!topk_merge_supported(n_parts * p->top_k, p->top_k)) return CSA_ERR_UNSUPPORTED;
     if (!cand_scores || !cand_ids || !part_ml || !workspace) return CSA_ERR_ARG;
     st = check_attn_ptrs(q, kv, kv_scales, p->kv_fmt, raw, n_raw, raw_pos0, q_pos, part_o, n_entries > 0);
     if (st) return st;
@@ -547,8 +548,10 @@ int csa_shard_attend(const csa_params* p, int32_t batch, const void* q, int32_t 
     const size_t sel_bytes = ((size_t(batch) * p->top_k * 4) + 255) & ~size_t(255);
     int32_t* sel_global = idx_out ? idx_out : (int32_t*)workspace;
     int32_t* sel_local = (int32_t*)((char*)workspace + sel_bytes);
+    // the merge's scratch and the attention's split partials share the space
+    // after the two selections (the merge is done before the attention starts)
     st = cuda_status(launch_topk_merge(batch, n_parts, p->top_k, cand_scores, cand_ids, entry0, n_entries,
-                                       sel_global, sel_local, s));
+                                       sel_global, sel_local, (char*)workspace + 2 * sel_bytes, p->m, p->window, s));
     if (st) return st;
     return run_attn(p, batch, 1, q, kv, kv_scales, n_entries, sel_local, raw, n_raw, raw_pos0, q_pos, nullptr,
                     part_o, (char*)workspace + 2 * sel_bytes, ws_bytes - 2 * sel_bytes,

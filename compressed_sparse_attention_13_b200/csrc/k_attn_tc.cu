@@ -79,7 +79,7 @@ struct SmemAttn {
     float alpha[kH], fin[kH];
     float2 ml[kH];                  // cluster combine: this split's (max in log2 units, sum) per head
     float cw[8][kH], cinv[kH];      // cluster combine: weight of each split, 1 / denominator
-    uint64_t raw_full[2], kv_full[2], kv_empty[2], s_full[2], p_full[2], o_done, q_full;
+    uint64_t raw_full[2], kv_half[2], kv_full[2], kv_empty[2], s_full[2], p_full[2], o_done, q_full;
     uint32_t tmem_base;
     int rescale;
 };
@@ -159,6 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.raw_full[i], 2);  // expect_tx arrival + arrival after the ids / scales
+            mbar_init(&S.kv_half[i], kConvWarps);  // one arrival per converter warp: dims 0..255 ready
             mbar_init(&S.kv_full[i], kConvWarps);  // one arrival per converter warp
             mbar_init(&S.kv_empty[i], 1);
             mbar_init(&S.s_full[i], 1);
@@ -168,8 +169,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&S.q_full, 1);
         S.rescale = 0;
         fence_mbar_init();
+        // the query's copy starts now, while TMEM is allocated and the CTA
+        // meets (this thread initialised its barrier)
+        prefetch_tmap(&map_win);
+        prefetch_tmap(&map_kv);
+        if (n_tiles > 0) {
+            mbar_arrive_expect_tx(&S.q_full, uint32_t(kH * kD * 2));
+#pragma unroll
+            for (int blk = 0; blk < 8; ++blk)
+                tma_load_2d(S.q[blk], &map_q, 64 * blk, int32_t(row * kH), &S.q_full);
+        }
     }
     if (warp == kMmaWarp) { tmem_alloc(&S.tmem_base, 512); tmem_relinquish(); }
+    // the issuer reads the first tile's selected ids before the CTA barrier
+    int32_t ids0[2] = {-1, -1};
+    if (warp == kIssuerWarp && n_tiles > 0) {
+        pdl_wait();  // the selected ids come from the kernel before this one
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int64_t slot = int64_t(tile0) * kTile + lane + 32 * h2;
+            ids0[h2] = (tile0 < kv_tiles && a.idx && slot < n_kv) ? a.idx[row * a.k + slot] : -1;
+        }
+    }
     pdl_launch_dependents();
     tc_fence_before();
     __syncthreads();
@@ -215,6 +236,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          S.kvs[kb][item][(128 * qt + 8 * c) >> 6]);
                         *reinterpret_cast<uint4*>(S.kv[kb][2 * qt + (c >> 3)] + sw128_offset(item, c & 7)) = o;
                     }
+                // the product over dims 0..255 may start while the upper half converts
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.kv_half[kb]);
                 // dims 256..511: read everything first, then overwrite the upper half
                 uint2 w[2][kUnits];
                 float sc[2][kUnits];
@@ -248,7 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async_smem();
             __syncwarp();  // the whole warp's tile writes are done: one arrival per warp
-            if (lane == 0) mbar_arrive(&S.kv_full[kb]);
+            if (lane == 0) {
+                if (!(kFp8 && tile0 + lt < kv_tiles)) mbar_arrive(&S.kv_half[kb]);
+                mbar_arrive(&S.kv_full[kb]);
+            }
         }
     } else if (warp == kIssuerWarp) {
         // ------------------------------------------------------------- issuer
@@ -256,13 +284,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n_tiles > 0) {
             const uint8_t* kv_seq = (const uint8_t*)a.kv + b * a.max_entries * int64_t(kFp8 ? kD : 0);
             const float* kvs_seq = (const float*)a.kv_s + b * a.max_entries * int64_t(kFp8 ? kD / 64 : 0);
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&S.q_full, uint32_t(kH * kD * 2));
-#pragma unroll
-                for (int blk = 0; blk < 8; ++blk)
-                    tma_load_2d(S.q[blk], &map_q, 64 * blk, int32_t(row * kH), &S.q_full);
-            }
-            pdl_wait();  // the selected ids come from the kernel before this one
             bool ok = true;
             int issued = 0;
             // software pipeline: the ids of tile lt+1 are loaded during tile lt,
@@ -275,8 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     j[h2] = (T < kv_tiles && a.idx && slot < n_kv) ? a.idx[row * a.k + slot] : -1;
                 }
             };
-            int32_t jn[2];
-            load_ids(0, jn);
+            int32_t jn[2] = {ids0[0], ids0[1]};  // tile 0's ids, read before the CTA barrier
 #pragma unroll 1
             for (int lt = 0; lt < n_tiles && ok; ++lt) {
                 const int kb = lt & 1, T = tile0 + lt;
@@ -385,23 +405,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             // which the softmax of tile t-2 has finished reading once P.V(t-2)
             // has been issued.  Each wait is a single non-blocking test; the
             // loop as a whole is bounded by kWaitNs without progress.
-            int qk_t = 0, pv_t = 0;
+            // QK of a tile runs in two halves over the dims: 0..255 once the
+            // converters have written them, 256..511 once the whole tile is in
+            int qk_t = 0, pv_t = 0, qk_half = 0;
             uint64_t t_last = global_ns();
             while (ok && pv_t < n_tiles) {
                 bool progressed = false;
                 if (qk_t < n_tiles && qk_t <= pv_t + 1) {
                     const int kb = qk_t & 1;
-                    if (mbar_test_wait(&S.kv_full[kb], uint32_t((qk_t >> 1) & 1))) {
+                    const uint32_t par = uint32_t((qk_t >> 1) & 1);
+                    if (mbar_test_wait(qk_half ? &S.kv_full[kb] : &S.kv_half[kb], par)) {
                         tc_fence_after();
                         const uint32_t kv0 = smem_u32(S.kv[kb][0]);
 #pragma unroll
-                        for (int s = 0; s < 32; ++s) {
-                            const int blk = s >> 2;
+                        for (int s = 0; s < 16; ++s) {
+                            const int blk = 4 * qk_half + (s >> 2);
                             mma_f16(tS + 64 * kb, smem_desc(q0 + blk * 8192 + (s & 3) * 32, 16, 1024),
-                                    smem_desc(kv0 + blk * 8192 + (s & 3) * 32, 16, 1024), id_qk, s != 0);
+                                    smem_desc(kv0 + blk * 8192 + (s & 3) * 32, 16, 1024), id_qk,
+                                    (qk_half | s) != 0);
                         }
-                        mma_commit(&S.s_full[kb]);
-                        ++qk_t;
+                        if (qk_half) {
+                            mma_commit(&S.s_full[kb]);
+                            ++qk_t;
+                        }
+                        qk_half ^= 1;
                         progressed = true;
                     }
                 }

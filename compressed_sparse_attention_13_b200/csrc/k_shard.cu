@@ -47,106 +47,115 @@ cudaError_t launch_shard_candidates(int64_t rows, int k, const float* scores, in
 
 namespace {
 
-constexpr int kMergeThreads = 1024;
-constexpr int kMergeCap = 16384;  // candidates per row (128 KB of 64-bit keys)
+constexpr int kMergeCap = 16384;   // candidates per row
+constexpr int kMapThreads = 1024;  // one CTA per row in the id mapping
 
-// Order-preserving map of an fp32 score to 32 bits (larger score, larger key).
-__device__ __forceinline__ uint32_t mono(float f) {
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+__global__ void gather_candidates_kernel(int64_t rows, int n_parts, int k, const float* __restrict__ cand_scores,
+                                         float* __restrict__ row_scores, int64_t* __restrict__ pos, int m, int W) {
+    const int64_t n = int64_t(n_parts) * k;
+    const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i < rows * n) {
+        const int64_t r = i / n, c = i - r * n;
+        row_scores[i] = cand_scores[((c / k) * rows + r) * k + c % k];
+    }
+    // the position whose eligible count is exactly the n candidates
+    if (i < rows) pos[i] = W + int64_t(m) * n;
 }
 
-// In-place bitonic sort, descending, of n (a power of two) 64-bit keys.
-__device__ void bitonic_desc(uint64_t* key, int n) {
-    for (int size = 2; size <= n; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            __syncthreads();
-            for (int i = threadIdx.x; i < (n >> 1); i += blockDim.x) {
-                const int lo = 2 * i - (i & (stride - 1));  // first of the pair
-                const int hi = lo + stride;
-                const bool desc = (lo & size) == 0;
-                const uint64_t a = key[lo], b = key[hi];
-                if ((a < b) == desc) { key[lo] = b; key[hi] = a; }
-            }
+// Exclusive prefix sum over the CTA (kMapThreads threads) of one value per
+// thread; returns this thread's offset and the total in *total.
+__device__ __forceinline__ int block_excl_scan(int v, int* total) {
+    __shared__ int warp_sum[kMapThreads / 32];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sum[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+        int w = lane < kMapThreads / 32 ? warp_sum[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
         }
+        warp_sum[lane] = w;  // inclusive prefix of the warp totals
     }
     __syncthreads();
+    const int before = (wid ? warp_sum[wid - 1] : 0) + x - v;
+    *total = warp_sum[kMapThreads / 32 - 1];
+    __syncthreads();  // warp_sum is reused by the next call
+    return before;
+}
+
+// Row r: the selected candidate positions (ascending) -> their global ids.
+// Positions ascend in (rank, slot) order, ranks hold increasing entry ranges
+// and each rank's candidates are in ascending id order, so the valid ids come
+// out ascending; empty candidates (-1) are dropped.
+__global__ void __launch_bounds__(kMapThreads) map_selection_kernel(
+    int64_t rows, int n_parts, int k, const int32_t* __restrict__ sel_pos, const int32_t* __restrict__ cand_ids,
+    int64_t entry0, int64_t n_entries, int32_t* __restrict__ sel_global, int32_t* __restrict__ sel_local) {
+    const int64_t r = blockIdx.x;
+    const int per = (k + kMapThreads - 1) / kMapThreads;  // consecutive slots per thread (<= 4)
+    const int i0 = threadIdx.x * per;
+    int32_t id[4];
+    int n_valid = 0, n_in = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        id[u] = -1;
+        if (u < per && i0 + u < k) {
+            const int32_t p = sel_pos[r * k + i0 + u];
+            if (p >= 0) id[u] = cand_ids[(int64_t(p / k) * rows + r) * k + p % k];
+        }
+        n_valid += id[u] >= 0;
+        n_in += id[u] >= entry0 && id[u] < entry0 + n_entries;
+    }
+    int tot_valid, tot_in;
+    int og = block_excl_scan(n_valid, &tot_valid);
+    int ol = block_excl_scan(n_in, &tot_in);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        if (id[u] < 0) continue;
+        sel_global[r * k + og++] = id[u];
+        if (id[u] >= entry0 && id[u] < entry0 + n_entries) sel_local[r * k + ol++] = int32_t(id[u] - entry0);
+    }
+    for (int i = tot_valid + threadIdx.x; i < k; i += kMapThreads) sel_global[r * k + i] = -1;
+    for (int i = tot_in + threadIdx.x; i < k; i += kMapThreads) sel_local[r * k + i] = -1;
 }
 
 }  // namespace
 
-// One CTA per row.  Valid candidates are keyed (mono(score) << 32) | ~id, so a
-// larger key is a higher score or, for equal scores, a smaller id; empty slots
-// are key 0, below every valid key (mono of any score is >= 0x007FFFFF).
-__global__ void __launch_bounds__(kMergeThreads) topk_merge_kernel(
-    int n_parts, int k, int64_t rows, const float* __restrict__ cand_scores, const int32_t* __restrict__ cand_ids,
-    int64_t entry0, int64_t n_entries, int32_t* __restrict__ sel_global, int32_t* __restrict__ sel_local) {
-    extern __shared__ uint64_t key[];
-    __shared__ int lo_cnt, hi_cnt;
-    const int64_t r = blockIdx.x;
-    const int n_cand = n_parts * k;
-    int n = 1;
-    while (n < n_cand) n <<= 1;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        uint64_t v = 0;
-        if (i < n_cand) {
-            const int64_t src = (int64_t(i / k) * rows + r) * k + i % k;
-            const int32_t id = cand_ids[src];
-            if (id >= 0) v = (uint64_t(mono(cand_scores[src])) << 32) | uint64_t(~uint32_t(id));
-        }
-        key[i] = v;
-    }
-    if (threadIdx.x == 0) { lo_cnt = 0; hi_cnt = 0; }
-    bitonic_desc(key, n);
-    // the first k keys are the selection; re-key them by id (ascending) and
-    // sort again: a valid entry becomes ~id (descending order = ascending
-    // id), an empty one 0 (last)
-    const int kk = min(k, n);
-    int n2 = 1;
-    while (n2 < kk) n2 <<= 1;
-    uint64_t* ids = key + n;  // scratch after the candidates (n2 <= n)
-    for (int i = threadIdx.x; i < n2; i += blockDim.x) {
-        uint64_t v = 0;
-        if (i < kk && key[i] != 0) v = uint64_t(uint32_t(key[i]));  // ~id: a larger key is a smaller id
-        ids[i] = v;
-    }
-    bitonic_desc(ids, n2);
-    // ascending ids; count those below entry0 and below entry0 + n_entries
-    int below_lo = 0, below_hi = 0;
-    for (int i = threadIdx.x; i < k; i += blockDim.x) {
-        const bool valid = i < kk && ids[i] != 0;
-        const int64_t id = valid ? int64_t(0xFFFFFFFFu - uint32_t(ids[i])) : -1;
-        sel_global[r * k + i] = int32_t(id);
-        if (valid && id < entry0) ++below_lo;
-        if (valid && id < entry0 + n_entries) ++below_hi;
-    }
-    atomicAdd(&lo_cnt, below_lo);
-    atomicAdd(&hi_cnt, below_hi);
-    __syncthreads();
-    const int a = lo_cnt, b = hi_cnt;
-    for (int i = threadIdx.x; i < k; i += blockDim.x) {
-        const int src = a + i;
-        sel_local[r * k + i] = src < b ? int32_t((0xFFFFFFFFu - uint32_t(ids[src])) - entry0) : -1;
-    }
-}
+bool topk_merge_supported(int n_cand, int k) { return n_cand > 0 && n_cand <= kMergeCap && k <= 4 * kMapThreads; }
 
-bool topk_merge_supported(int n_cand) { return n_cand > 0 && n_cand <= kMergeCap; }
-// (k <= 4096 keeps the candidates and the re-keyed selection within 160 KB)
+size_t topk_merge_workspace(int64_t rows, int k) {
+    const size_t sc = (size_t(rows) * kMergeCap * 4 + 255) & ~size_t(255);
+    const size_t ps = (size_t(rows) * 8 + 255) & ~size_t(255);
+    const size_t sp = (size_t(rows) * k * 4 + 255) & ~size_t(255);
+    return sc + ps + sp;
+}
 
 cudaError_t launch_topk_merge(int64_t rows, int n_parts, int k, const float* cand_scores, const int32_t* cand_ids,
                               int64_t entry0, int64_t n_entries, int32_t* sel_global, int32_t* sel_local,
-                              cudaStream_t s) {
+                              void* ws, int m, int W, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
     const int n_cand = n_parts * k;
-    if (!topk_merge_supported(n_cand)) return cudaErrorInvalidValue;
-    int n = 1;
-    while (n < n_cand) n <<= 1;
-    int n2 = 1;
-    while (n2 < std::min(k, n)) n2 <<= 1;
-    const size_t sm = size_t(n + n2) * sizeof(uint64_t);
-    cudaError_t e = ensure_smem(topk_merge_kernel, sm);
+    if (!topk_merge_supported(n_cand, k)) return cudaErrorInvalidValue;
+    // the candidates of a row side by side: the top-k over positions, ties
+    // to the lower position, is the top-k by score then id
+    float* row_scores = (float*)ws;
+    int64_t* pos = (int64_t*)((char*)ws + ((size_t(rows) * kMergeCap * 4 + 255) & ~size_t(255)));
+    int32_t* sel_pos = (int32_t*)((char*)pos + ((size_t(rows) * 8 + 255) & ~size_t(255)));
+    const int64_t n = rows * n_cand;
+    gather_candidates_kernel<<<unsigned(ceil_div(std::max<int64_t>(n, rows), 256)), 256, 0, s>>>(
+        rows, n_parts, k, cand_scores, row_scores, pos, m, W);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    topk_merge_kernel<<<unsigned(rows), kMergeThreads, sm, s>>>(n_parts, k, rows, cand_scores, cand_ids, entry0,
+    e = launch_topk(row_scores, n_cand, n_cand, pos, m, W, k, rows, sel_pos, s);
+    if (e != cudaSuccess) return e;
+    map_selection_kernel<<<unsigned(rows), kMapThreads, 0, s>>>(rows, n_parts, k, sel_pos, cand_ids, entry0,
                                                                 n_entries, sel_global, sel_local);
     return cudaGetLastError();
 }

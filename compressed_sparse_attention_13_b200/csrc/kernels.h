@@ -90,9 +90,13 @@ cudaError_t launch_shard_candidates(int64_t rows, int k, const float* scores, in
 // ranked by score and then by the smaller id; writes the selection as
 // ascending global ids (-1 padded) and the part in [entry0, entry0 + n_entries)
 // as ascending local ids (-1 padded).
-bool topk_merge_supported(int n_cand);
+// ws: topk_merge_workspace(rows, k) bytes (candidate rows, positions, the
+// selected positions); m, W: the layer's, for the eligibility rule the top-k
+// kernels apply.
+bool topk_merge_supported(int n_cand, int k);
+size_t topk_merge_workspace(int64_t rows, int k);
 cudaError_t launch_topk_merge(int64_t rows, int n_parts, int k, const float* cand_scores, const int32_t* cand_ids,
                               int64_t entry0, int64_t n_entries, int32_t* sel_global, int32_t* sel_local,
-                              cudaStream_t s);
+                              void* ws, int m, int W, cudaStream_t s);
 
 }  // namespace csa

@@ -88,6 +88,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     return false;
 }
 
+// Fetch a tensor map (a __grid_constant__ kernel parameter) into the TMA
+// unit's descriptor cache ahead of its first copy.
+__device__ __forceinline__ void prefetch_tmap(const void* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
 // ------------------------------------------------------------ bulk copies
 // 1-D bulk copy global -> shared, completing `bytes` of transaction on bar.
 // Both addresses 16-byte aligned, bytes a multiple of 16.
