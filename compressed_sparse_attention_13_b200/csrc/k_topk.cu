@@ -4,11 +4,12 @@
 // Every kernel here ranks the order-preserving 32-bit image of each fp32 score
 // (-0.0 folded into +0.0), finds the exact k-th largest key T by radix passes
 // and how many keys equal to T are taken, and writes the selected ids in
-// ascending order, ties going to the lower index.  Rows of up to 32,768
-// scores (decode at 128K context, prefill chunks) take topk_sel_kernel, which
-// narrows the row to a few times k candidates with a sampled threshold
-// first; longer rows take a thread-block cluster per row (few rows) or one
-// CTA per row reading the row from global memory (many rows).
+// ascending order, ties going to the lower index.  Many rows of up to 2,048
+// scores (prefill chunks) take one warp per row; rows of up to 32,768 scores
+// (decode at 128K context) take topk_sel_kernel, which narrows the row to a
+// few times k candidates with a sampled threshold first; longer rows take a
+// thread-block cluster per row (few rows) or one CTA per row reading the row
+// from global memory (many rows).
 #include <cooperative_groups.h>
 
 #include "kernels.h"
@@ -248,6 +249,101 @@ __global__ void __launch_bounds__(kTopkThreads) topk_smem_kernel(
         __syncthreads();
     }
     write_selection_impl([&](int64_t i) { return keys[i]; }, int64_t(n), prefix, remaining, k, out, warp_tot);
+}
+
+// Many short rows (prefill chunks: up to 2,048 scores per row): one warp per
+// row with the row in registers (lane l holds keys l + 32 i), so the four
+// radix passes and the ordered output synchronise only the warp.  Each pass
+// counts the keys that match the prefix so far into the warp's 256-bin
+// shared histogram, lanes holding the same digit merged by __match_any_sync
+// (N(0, s) scores share a few exponent digits); the output walks the row 32
+// consecutive keys at a time, compacting with ballots.
+constexpr int kWarpRowMax = 2048;
+constexpr int kWarpRowThreads = 128;  // 4 rows per CTA
+
+__global__ void __launch_bounds__(kWarpRowThreads) topk_warp_kernel(
+    const float* __restrict__ scores, int64_t ld, int64_t max_blocks, const int64_t* __restrict__ q_pos, int m,
+    int W, int k, int64_t rows, int32_t* __restrict__ idx) {
+    constexpr int kPer = kWarpRowMax / 32;
+    __shared__ int hist[kWarpRowThreads / 32][256];
+    pdl_wait();  // the scores come from the kernel before this one
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+    const int64_t row = int64_t(blockIdx.x) * (kWarpRowThreads / 32) + wl;
+    if (row >= rows) return;  // whole warps leave together
+    const float* s = scores + row * ld;
+    int32_t* out = idx + row * k;
+    const int n = int(min(n_elig(q_pos[row], m, W), max_blocks));
+    if (n <= k) {
+        for (int i = lane; i < k; i += 32) out[i] = i < n ? i : -1;
+        return;
+    }
+    uint32_t key[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int e = 32 * i + lane;
+        key[i] = e < n ? order_key(s[e]) : 0u;
+    }
+    int* h = hist[wl];
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = k;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int j = lane; j < 256; j += 32) h[j] = 0;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            if (32 * i >= n) break;  // uniform across the warp
+            const int e = 32 * i + lane;
+            const bool in = e < n && (key[i] & pmask) == prefix;
+            const uint32_t dg = in ? ((key[i] >> shift) & 255u) : 0xFFFFFFFFu;
+            const unsigned same = __match_any_sync(0xffffffffu, dg);
+            if (in && lane == __ffs(same) - 1) h[dg] += __popc(same);
+        }
+        __syncwarp();
+        // lane l owns the 8 bins counted from the top: 255-8l .. 248-8l
+        int loc[8], sum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { loc[j] = h[255 - 8 * lane - j]; sum += loc[j]; }
+        int inc = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        int above = inc - sum, fd = -1, fa = 0;
+        if (above < remaining && remaining <= inc) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (above < remaining && remaining <= above + loc[j]) { fd = 255 - 8 * lane - j; fa = above; }
+                above += loc[j];
+            }
+        }
+        const int src = __ffs(__ballot_sync(0xffffffffu, fd >= 0)) - 1;
+        fd = __shfl_sync(0xffffffffu, fd, src);
+        fa = __shfl_sync(0xffffffffu, fa, src);
+        remaining -= fa;
+        prefix |= uint32_t(fd) << shift;
+        pmask |= 0xFFu << shift;
+        __syncwarp();
+    }
+    // every key above T = prefix, then the first `remaining` keys equal to T
+    const unsigned lt = (1u << lane) - 1u;
+    int pos = 0, eq_before = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        if (32 * i >= n) break;
+        const int e = 32 * i + lane;
+        const bool valid = e < n;
+        const bool is_eq = valid && key[i] == prefix;
+        const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+        const bool take = valid && (key[i] > prefix || (is_eq && eq_before + __popc(eqm & lt) < remaining));
+        const unsigned tm = __ballot_sync(0xffffffffu, take);
+        if (take) out[pos + __popc(tm & lt)] = e;
+        pos += __popc(tm);
+        eq_before += __popc(eqm);
+    }
 }
 
 // Few rows (decode): one thread-block cluster of kClu CTAs per row (rows of
@@ -890,6 +986,9 @@ cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, con
     // (many short rows -- a prefill chunk -- are faster with the whole row in
     // one CTA's shared memory and no sampling: topk_smem_kernel below)
     const bool many_short = rows >= 2 * kNumSMs && max_blocks <= 4096;
+    if (many_short && max_blocks <= kWarpRowMax)
+        return launch_ex(topk_warp_kernel, dim3(unsigned(ceil_div(rows, kWarpRowThreads / 32))),
+                         dim3(kWarpRowThreads), 0, s, pdl, scores, ld, max_blocks, q_pos, m, W, k, rows, idx);
     if (k <= kSelCap / 2 && rows * 8 <= INT32_MAX && max_blocks <= INT32_MAX / 2 && !many_short) {
         if (max_blocks <= 2048) return launch_topk_sel<1, 1>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
         if (max_blocks <= 8192) return launch_topk_sel<1, 4>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);

@@ -168,14 +168,17 @@ def test_indexer_matches_oracle(idx, HI, dI, n_q, nb, m, W):
 
 
 # --------------------------------------------------------------------- top-k
-# Few rows take the cluster kernel (one 8-CTA cluster per row, up to 294,912
-# scores); many rows, or longer rows, take one CTA per row with the row in
-# shared memory (up to 45056 scores) or read from global memory.
+# Up to 32,768 scores: the sampled-threshold kernel (1, 4 or 8 CTAs per row);
+# longer rows: a cluster per row (few rows) or one CTA per row reading the
+# row from global memory; many rows (>= 296) of up to 2,048 scores: one warp
+# per row; of up to 4,096: one CTA per row in shared memory.
 @pytest.mark.parametrize("n,k,rows", [
-    (50, 8, 6), (2015, 512, 6), (32736, 512, 6), (5000, 1024, 6), (60000, 1024, 6),  # cluster
-    (2015, 512, 48), (32736, 512, 48),                                                 # shared memory
-    (70000, 1024, 6), (250000, 1024, 6),                                              # cluster, large
-    (60000, 1024, 40), (300000, 512, 6),                                               # global
+    (50, 8, 6), (2015, 512, 6), (32736, 512, 6), (5000, 1024, 6), (60000, 1024, 6),
+    (2015, 512, 48), (32736, 512, 48),
+    (70000, 1024, 6), (250000, 1024, 6),
+    (60000, 1024, 40), (300000, 512, 6),
+    (2016, 512, 300), (2048, 1024, 301), (700, 64, 400),                              # warp per row
+    (4000, 512, 300),                                                                  # shared memory
 ])
 def test_topk_matches_oracle_exactly(n, k, rows):
     s = synth.tensor_np(4, "ts", (rows, n))
