@@ -764,6 +764,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     __shared__ int sh[4];
     __shared__ int s_count;
     __shared__ int s_bin[CPR];
+    __shared__ int s_woff[kSelThreads / 32], s_base;
     pdl_wait();  // the scores come from the kernel before this one
     pdl_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31;
@@ -851,14 +852,29 @@ __global__ void __launch_bounds__(kSelThreads, 1)
             if constexpr (CPR > 1) cluster_wait_acquire();
             else __syncthreads();
         }
-        // 2. candidates into the leader: a per-warp count, one reservation per warp
+        // 2. candidates into the leader: per-warp counts, scanned in the CTA,
+        // and one reservation in the leader per CTA and batch (remote atomics
+        // on one counter serialise, so there are as few as possible)
         int cnt = 0;
 #pragma unroll
         for (int j = 0; j < 4 * V; ++j)
             cnt += __popc(__ballot_sync(0xffffffffu, key[j] != 0u && int(key[j] >> kSelBinShift) >= b_r));
-        int slot = 0;
-        if (lane == 0 && cnt) slot = atomicAdd(lcount, cnt);
-        slot = __shfl_sync(0xffffffffu, slot, 0);
+        if (lane == 0) s_woff[tid >> 5] = cnt;
+        __syncthreads();
+        if (tid < 32) {
+            const int v = tid < kSelThreads / 32 ? s_woff[tid] : 0;
+            int inc = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, inc, o);
+                if (tid >= o) inc += y;
+            }
+            const int total = __shfl_sync(0xffffffffu, inc, 31);
+            if (tid < kSelThreads / 32) s_woff[tid] = inc - v;
+            if (tid == 0) s_base = total ? atomicAdd(lcount, total) : 0;
+        }
+        __syncthreads();
+        int slot = s_base + s_woff[tid >> 5];
 #pragma unroll
         for (int j = 0; j < 4 * V; ++j) {
             const bool c = key[j] != 0u && int(key[j] >> kSelBinShift) >= b_r;
@@ -916,20 +932,35 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         if (take) atomicOr(&bitmap[ci[i] >> 5], 1u << (ci[i] & 31u));
     }
     __syncthreads();
-    const int per = (words + kSelThreads - 1) / kSelThreads;
-    const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+    // warp w owns a contiguous range of 32-word chunks; lane l reads word l of
+    // a chunk (no bank conflicts), a warp scan of the words' counts places them
+    constexpr int kWarps = kSelThreads / 32;
+    const int wid = tid >> 5;
+    const int wpw = ((words + kWarps - 1) / kWarps + 31) & ~31;  // words per warp
+    const int w0 = min(words, wid * wpw), w1 = min(words, w0 + wpw);
     int c = 0;
-    for (int wi = w0; wi < w1; ++wi) c += __popc(bitmap[wi]);
-    const int2 incl = block_scan2<kSelThreads>(make_int2(c, 0), warp_tot);
-    int pos = incl.x - c;
-    for (int wi = w0; wi < w1; ++wi) {
-        uint32_t b = bitmap[wi];
+    for (int wi = w0 + lane; wi < w1; wi += 32) c += __popc(bitmap[wi]);
+    const int wc = __reduce_add_sync(0xffffffffu, c);  // every lane takes part
+    const int2 incl = block_scan2<kSelThreads>(make_int2(lane == 0 ? wc : 0, 0), warp_tot);
+    int pos = __shfl_sync(0xffffffffu, incl.x, 0) - wc;
+    for (int cb = w0; cb < w1; cb += 32) {
+        const int wi = cb + lane;
+        uint32_t b = wi < w1 ? bitmap[wi] : 0u;
+        const int pc = __popc(b);
+        int inc = pc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        int p = pos + inc - pc;
         while (b) {
             const int bit = __ffs(b) - 1;
             b &= b - 1;
-            if (pos < k) out[pos] = wi * 32 + bit;
-            ++pos;
+            if (p < k) out[p] = wi * 32 + bit;
+            ++p;
         }
+        pos += __shfl_sync(0xffffffffu, inc, 31);
     }
 }
 
@@ -943,6 +974,10 @@ static cudaError_t launch_topk_sel(const float* scores, int64_t ld, int64_t max_
     const size_t sm = (2 * size_t(cap) + size_t((max_blocks + 31) / 32)) * 4;
     cudaError_t e = ensure_smem(topk_sel_kernel<CPR, V>, sm);
     if (e != cudaSuccess) return e;
+    if (CPR > 8) {  // clusters beyond the portable 8 CTAs
+        e = cudaFuncSetAttribute(topk_sel_kernel<CPR, V>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
     const int vec = ((reinterpret_cast<uintptr_t>(scores) & 15) == 0 && (ld % 4) == 0) ? 1 : 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(rows * CPR));
@@ -965,6 +1000,23 @@ static cudaError_t launch_topk_sel(const float* scores, int64_t ld, int64_t max_
     }
     cfg.attrs = na ? attr : nullptr;
     cfg.numAttrs = na;
+    if (CPR > 8) {
+        // a 16-CTA cluster needs 16 free SMs of one GPC; fall back when the
+        // device cannot place one (queried once per device)
+        static int known[64];  // 0 unknown, 1 yes, 2 no
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidValue;
+        if (known[dev] == 0) {
+            int n_clusters = 0;
+            cudaLaunchConfig_t q = cfg;
+            q.numAttrs = 1;  // the cluster dimension alone
+            const bool ok = cudaOccupancyMaxActiveClusters(&n_clusters, topk_sel_kernel<CPR, V>, &q) == cudaSuccess &&
+                            n_clusters > 0;
+            if (!ok) (void)cudaGetLastError();
+            known[dev] = ok ? 1 : 2;
+        }
+        if (known[dev] == 2) return cudaErrorNotSupported;
+    }
     return cudaLaunchKernelEx(&cfg, topk_sel_kernel<CPR, V>, scores, ld, max_blocks, q_pos, m, W, k, idx, seg,
                               cap, vec);
 }
@@ -993,6 +1045,11 @@ cudaError_t launch_topk(const float* scores, int64_t ld, int64_t max_blocks, con
         if (max_blocks <= 2048) return launch_topk_sel<1, 1>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
         if (max_blocks <= 8192) return launch_topk_sel<1, 4>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
         if (max_blocks <= 32768) return launch_topk_sel<4, 4>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
+        if (max_blocks > 65536 && rows * 16 <= kNumSMs) {
+            // few long rows (a 1M-token sequence): 16 CTAs per row, one batch each
+            const cudaError_t e = launch_topk_sel<16, 8>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
+            if (e != cudaErrorNotSupported) return e;
+        }
         return launch_topk_sel<8, 8>(scores, ld, max_blocks, q_pos, m, W, k, rows, idx, s, pdl);
     }
     // Few longer rows cannot fill the GPU with one CTA each: give each row a cluster.
