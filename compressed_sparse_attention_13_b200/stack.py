@@ -49,7 +49,10 @@ class Layer:
         self.spec = spec
         p = spec.p
         self.m, self.W, self.d = p.m, p.window, p.head_dim
-        self.cap_blocks = (spec.prior_tokens + spec.new_tokens) // self.m
+        # capacity in whole 128-row steps: the tensor-core MXFP4 indexer takes
+        # a row count that is a multiple of 4 (rows past the pooled ones are
+        # never read: only n_elig(t) entries are visible)
+        self.cap_blocks = -(-((spec.prior_tokens + spec.new_tokens) // self.m) // 128) * 128
         # the window-only block keeps no pooled cache
         self.kv = empty_stored(FP8_S64, self.cap_blocks, self.d, device) if spec.kind != "window" else None
         self.kI = empty_stored(MXFP4, self.cap_blocks, p.idx_dim, device) if spec.kind == "csa" else None

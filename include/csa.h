@@ -166,9 +166,12 @@ int csa_quantize(int32_t fmt, const float* src, int64_t rows, int32_t d, void* o
  *   kI:        [batch][max_blocks][dI] in p->idx_fmt (+ kI_scales)
  *   q_pos:     int64 [batch][n_q]
  *   scores:    float [batch][n_q][ld_scores], ld_scores >= max_blocks
- * Formats without a tensor-core path (F32, and BF16 with fewer than 4
- * queries per sequence) take at most 65535 query rows (batch * n_q) per
- * call; larger calls return CSA_ERR_UNSUPPORTED.
+ * The tensor-core kernels take MXFP4 with HI = 64, dI = 128, max_blocks a
+ * multiple of 4 and batch * max_blocks >= 128, and BF16 with at least 4
+ * queries per sequence; other calls run on the CUDA cores (much slower at
+ * long contexts: allocate max_blocks in multiples of 4).  Formats without a
+ * tensor-core path take at most 65535 query rows (batch * n_q) per call;
+ * larger calls return CSA_ERR_UNSUPPORTED.
  * ------------------------------------------------------------------------ */
 int indexer_score(const csa_params* p, int32_t batch, int32_t n_q, const void* qI,
                   const void* qI_scales, const float* w, const void* kI, const void* kI_scales,

@@ -67,18 +67,19 @@ class _Draw:
         return _bf16_host(t) if t.dtype == torch.bfloat16 else t.detach().cpu().numpy()
 
 
-def _run_layer(kind, g, prior, chunk, steps, topk):
+def _run_layer(kind, g, prior, chunk, steps, topk, win=W):
     """Run one layer (prior cache, chunk, decode steps) on the device; returns
     the outputs and selections of the chunk and of the decode steps, and the
     layer's caches."""
     m = 128 if kind == "hca" else 4
-    p = K.params(m, W, topk if kind == "csa" else 1, H, D, HI, DI, SCALE, K.BF16, K.FP8_S64, K.MXFP4)
+    p = K.params(m, win, topk if kind == "csa" else 1, H, D, HI, DI, SCALE, K.BF16, K.FP8_S64, K.MXFP4)
     n_new = chunk + steps
     L = Layer(LayerSpec(kind, p, prior, n_new))
     if kind != "window":
         K.csa_quantize(g("prior_kv", (prior // m, D)), K.Stored(K.FP8_S64, L.kv.data[:prior // m],
                                                                 L.kv.scales[:prior // m]))
-    L.set_prior_window(g("x_prior", (W - 1, D), dt="bf16"))
+    if win > 1:
+        L.set_prior_window(g("x_prior", (win - 1, D), dt="bf16"))
     x, z = g("x", (n_new, D), dt="bf16"), g("z", (n_new, D), dt="bf16")
     bias, q, sinks = g("bias", (m, D), 0.1), g("q", (n_new, H, D), dt="bf16"), g("sinks", (H,))
     out = torch.empty(n_new, H, D, dtype=torch.bfloat16, device="cuda")
@@ -145,11 +146,12 @@ def _oracle_caches(kind, g, res, prior, n_pooled_new):
     return caches
 
 
-def _check_rows(kind, g, res, caches, prior, check_rows, topk):
+def _check_rows(kind, g, res, caches, prior, check_rows, topk, win=W):
     """Outputs (and CSA selections) of the given new-token rows against the oracle."""
     m = res["m"]
-    raw = oracle.Stored(oracle.BF16, np.concatenate([g.host("x_prior"), g.host("x")]))
-    raw_pos0 = prior - (W - 1)
+    W = win  # noqa: N806 (the window of this layer)
+    raw = oracle.Stored(oracle.BF16, np.concatenate([g.host("x_prior"), g.host("x")]) if W > 1 else g.host("x"))
+    raw_pos0 = prior - (W - 1) if W > 0 else prior
     q = g.host("q")
     sinks = g.host("sinks")
     rows = np.asarray(check_rows, np.int64)
@@ -214,3 +216,15 @@ def test_interleaved_stack_full_size_sampled_rows():
         _check_rows(kind, g, res, caches, prior, rows, topk)
         del res, caches, g
         torch.cuda.empty_cache()
+
+
+def test_csa_layer_without_window():
+    """W = 0: no raw window at all; the prefill's raw buffer starts at the
+    chunk (t0) and the decode steps attend to pooled entries only."""
+    prior, topk, chunk, steps = 2048, 128, 256, 16
+    K.csa_device_status(reset=True)
+    g = _Draw("stack/nowin", 47)
+    res = _run_layer("csa", g, prior, chunk, steps, topk, win=0)
+    caches = _oracle_caches("csa", g, res, prior, (chunk + steps) // 4)
+    rows = sorted(set(range(0, chunk, 41)) | {chunk - 1} | set(range(chunk, chunk + steps)))
+    _check_rows("csa", g, res, caches, prior, rows, topk, win=0)
