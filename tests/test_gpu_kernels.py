@@ -70,6 +70,10 @@ def test_quantize_bf16_matches_oracle():
     ("bf16", 4, 512, 97, "f32"),
     ("bf16", 128, 512, 5, "f32"),
     ("f32", 4, 128, 33, "f32"),
+    # m a multiple of 16: the staged kernel (bulk copies through shared memory)
+    ("f32", 128, 512, 7, "f32"),
+    ("bf16", 32, 256, 300, "f32"),        # more rows than CTAs
+    ("bf16", 16, 64, 9, "f32"),
 ])
 def test_compress_f32_out(act, m, d, n_blocks, out):
     n = m * n_blocks
@@ -88,6 +92,9 @@ def test_compress_f32_out(act, m, d, n_blocks, out):
     ("bf16", 128, 512, 6, "fp8"),
     ("bf16", 4, 512, 40, "bf16"),
     ("f32", 4, 128, 70, "mxfp4"),
+    ("bf16", 128, 512, 600, "fp8"),       # staged kernel, several rows per CTA
+    ("bf16", 16, 128, 50, "mxfp4"),
+    ("f32", 64, 512, 5, "bf16"),
 ])
 def test_compress_quantised_out(act, m, d, n_blocks, fmt):
     n = m * n_blocks
