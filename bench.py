@@ -1099,6 +1099,31 @@ def run_case(name, reps=3):
         q_pos = torch.arange(T, dtype=torch.int64, device=dev)
         sel = torch.empty(T, w.k, dtype=torch.int32, device=dev)
         fn = lambda: K.topk_select(p, 1, T, scores, nb, nb, q_pos, sel)
+    elif name == "decode_128k_b32_fp8_indexer":   # the indexer's exact E2M1 -> E4M3 variant on C2
+        w = WORKLOADS[WORKLOAD]
+        S = setup_csa_decode(w, dev)
+        S["p"] = K.params(w.m, w.W, w.k, w.H, w.d, w.HI, w.dI, w.scale, K.BF16, K.FP8_S64, K.MXFP4,
+                          flags=K.FLAG_INDEXER_FP8)
+        fn = lambda: csa_decode_call(w, S)
+    elif name == "prefill_8k_attn":     # the bf16 prefill's attention stage (8192 rows, bf16 entries)
+        w = WORKLOADS["csa_prefill_8k_bf16"]
+        T, nb, H, d = w.n_ctx, w.n_ctx // w.m, w.H, w.d
+        p = K.params(w.m, w.W, w.k, H, d, w.HI, w.dI, w.scale, K.BF16, K.BF16, K.BF16)
+        kv = K.Stored(K.BF16, tensor_torch(0, "case/pa/kv", (nb, d), dtype="bf16", device=dev))
+        q = tensor_torch(0, "case/pa/q", (T, H, d), dtype="bf16", device=dev)
+        raw = tensor_torch(0, "case/pa/x", (1, T, d), dtype="bf16", device=dev)
+        sinks = tensor_torch(0, "case/pa/sinks", (H,), device=dev)
+        q_pos = torch.arange(T, dtype=torch.int64, device=dev)
+        # a valid selection: the k most recent eligible entries of each row
+        e = torch.arange(w.k, device=dev)[None, :]
+        ne = torch.clamp((q_pos[:, None] - w.W) // w.m, min=0)
+        idx = torch.where(e < ne, ne - 1 - e, torch.full_like(e, -1)).flip(1).to(torch.int32)
+        idx = torch.sort(torch.where(idx < 0, torch.full_like(idx, 1 << 30), idx), dim=1).values
+        idx = torch.where(idx == (1 << 30), torch.full_like(idx, -1), idx).contiguous()
+        out = torch.empty(T, H, d, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(K.csa_workspace_size(p, K.OP_SPARSE_ATTN, 1, T, 0), dtype=torch.uint8, device=dev)
+        pos0 = torch.zeros(1, dtype=torch.int64, device=dev)
+        fn = lambda: K.sparse_mqa_attn(p, 1, T, q, kv, nb, idx, raw, T, pos0, q_pos, sinks, out, ws)
     else:
         raise SystemExit(f"unknown case {name}")
     torch.cuda.empty_cache()   # only the case's own tensors stay on the device
