@@ -114,7 +114,8 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
                     const void* kv_s, int64_t max_entries, const int32_t* idx, const void* raw,
                     int64_t n_raw, const int64_t* raw_pos0, const int64_t* q_pos,
                     const float* sinks, void* out, void* ws, size_t ws_bytes, int64_t items_per_row,
-                    cudaStream_t s, bool pdl = false, float2* part_ml = nullptr, int64_t kv_base = 0) {
+                    cudaStream_t s, bool pdl = false, float2* part_ml = nullptr, int64_t kv_base = 0,
+                    const int32_t* n_sel = nullptr) {
     const int64_t rows = int64_t(batch) * n_q;
     if (!attn_simt_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim) &&
         !attn_tc_supported(p->act_fmt, p->kv_fmt, p->n_heads, p->head_dim))
@@ -132,6 +133,7 @@ static int run_attn(const csa_params* p, int batch, int n_q, const void* q, cons
     a.part_ml = (float2*)((char*)ws + plan.part_o_bytes);
     a.partial_out = part_ml != nullptr;
     a.kv_base = kv_base;
+    a.n_sel = n_sel;
     if (part_ml && plan.n_splits == 1) {  // the one split's partial is the result
         a.part_o = (float*)out;
         a.part_ml = part_ml;
@@ -366,8 +368,9 @@ size_t csa_workspace_size(const csa_params* p, int32_t op, int32_t batch, int64_
     }
     case CSA_OP_SHARD_ATTEND: {
         const size_t sel = ((size_t(rows) * p->top_k * 4) + 255) & ~size_t(255);
+        const size_t cnt = ((size_t(rows) * 4) + 255) & ~size_t(255);
         const size_t merge = topk_merge_workspace(rows, p->top_k);
-        return 2 * sel + std::max(merge, plan_attn(p, rows, int64_t(p->top_k) + p->window).bytes()) + 256;
+        return 2 * sel + cnt + std::max(merge, plan_attn(p, rows, int64_t(p->top_k) + p->window).bytes()) + 256;
     }
     case CSA_OP_HCA_SHARD:
         return plan_attn(p, rows, n_ctx + p->window).bytes() + 256;
@@ -546,16 +549,21 @@ int csa_shard_attend(const csa_params* p, int32_t batch, const void* q, int32_t 
     if (ws_bytes < csa_workspace_size(p, CSA_OP_SHARD_ATTEND, batch, 1, n_entries)) return CSA_ERR_WORKSPACE;
     const cudaStream_t s = (cudaStream_t)stream;
     const size_t sel_bytes = ((size_t(batch) * p->top_k * 4) + 255) & ~size_t(255);
+    const size_t cnt_bytes = ((size_t(batch) * 4) + 255) & ~size_t(255);
     int32_t* sel_global = idx_out ? idx_out : (int32_t*)workspace;
     int32_t* sel_local = (int32_t*)((char*)workspace + sel_bytes);
+    int32_t* n_local = (int32_t*)((char*)workspace + 2 * sel_bytes);
+    char* rest = (char*)workspace + 2 * sel_bytes + cnt_bytes;
+    const size_t rest_bytes = ws_bytes - 2 * sel_bytes - cnt_bytes;
     // the merge's scratch and the attention's split partials share the space
-    // after the two selections (the merge is done before the attention starts)
+    // after the selections (the merge is done before the attention starts)
     st = cuda_status(launch_topk_merge(batch, n_parts, p->top_k, cand_scores, cand_ids, entry0, n_entries,
-                                       sel_global, sel_local, (char*)workspace + 2 * sel_bytes, p->m, p->window, s));
+                                       sel_global, sel_local, n_local, rest, p->m, p->window, s));
     if (st) return st;
+    // the local selection is compacted: the attention visits only its n_local slots
     return run_attn(p, batch, 1, q, kv, kv_scales, n_entries, sel_local, raw, n_raw, raw_pos0, q_pos, nullptr,
-                    part_o, (char*)workspace + 2 * sel_bytes, ws_bytes - 2 * sel_bytes,
-                    int64_t(p->top_k) + p->window, s, false, (float2*)part_ml);
+                    part_o, rest, rest_bytes, int64_t(p->top_k) + p->window, s, false, (float2*)part_ml, 0,
+                    n_local);
 }
 
 int hca_shard_attend(const csa_params* p, int32_t batch, const void* q, const void* kv, const void* kv_scales,

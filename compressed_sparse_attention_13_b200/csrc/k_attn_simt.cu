@@ -32,7 +32,8 @@ __device__ __forceinline__ RowSlots row_slots(const AttnArgs& a, int64_t row) {
     RowSlots r;
     const int64_t b = row / a.n_q;
     const int64_t t = a.q_pos[row];
-    r.n_kv = a.idx ? a.k : min(max(n_elig(t, a.m, a.W) - a.kv_base, int64_t(0)), a.max_entries);
+    r.n_kv = a.idx ? (a.n_sel ? min(int64_t(a.n_sel[row]), int64_t(a.k)) : a.k)
+                   : min(max(n_elig(t, a.m, a.W) - a.kv_base, int64_t(0)), a.max_entries);
     const int64_t p0 = a.raw_pos0[b];
     const int64_t lo = max(max(t - a.W + 1, int64_t(0)), p0);
     const int64_t hi = min(t + 1, p0 + a.n_raw);

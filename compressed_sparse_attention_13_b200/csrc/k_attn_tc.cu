@@ -146,7 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int split = blockIdx.x;
     const int64_t b = row / a.n_q;
     const int64_t t = a.q_pos[row];
-    const int64_t n_kv = a.idx ? a.k : min(max(n_elig(t, a.m, a.W) - a.kv_base, int64_t(0)), a.max_entries);
+    const int64_t n_kv = a.idx ? (a.n_sel ? min(int64_t(a.n_sel[row]), int64_t(a.k)) : a.k)
+                               : min(max(n_elig(t, a.m, a.W) - a.kv_base, int64_t(0)), a.max_entries);
     const int64_t p0 = a.raw_pos0[b];
     const int64_t win_lo = max(max(t - a.W + 1, int64_t(0)), p0);
     const int64_t n_win = max(int64_t(0), min(t + 1, p0 + a.n_raw) - win_lo);

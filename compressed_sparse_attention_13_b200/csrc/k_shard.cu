@@ -97,7 +97,8 @@ __device__ __forceinline__ int block_excl_scan(int v, int* total) {
 // out ascending; empty candidates (-1) are dropped.
 __global__ void __launch_bounds__(kMapThreads) map_selection_kernel(
     int64_t rows, int n_parts, int k, const int32_t* __restrict__ sel_pos, const int32_t* __restrict__ cand_ids,
-    int64_t entry0, int64_t n_entries, int32_t* __restrict__ sel_global, int32_t* __restrict__ sel_local) {
+    int64_t entry0, int64_t n_entries, int32_t* __restrict__ sel_global, int32_t* __restrict__ sel_local,
+    int32_t* __restrict__ n_local) {
     const int64_t r = blockIdx.x;
     const int per = (k + kMapThreads - 1) / kMapThreads;  // consecutive slots per thread (<= 4)
     const int i0 = threadIdx.x * per;
@@ -124,6 +125,7 @@ __global__ void __launch_bounds__(kMapThreads) map_selection_kernel(
     }
     for (int i = tot_valid + threadIdx.x; i < k; i += kMapThreads) sel_global[r * k + i] = -1;
     for (int i = tot_in + threadIdx.x; i < k; i += kMapThreads) sel_local[r * k + i] = -1;
+    if (threadIdx.x == 0) n_local[r] = tot_in;
 }
 
 }  // namespace
@@ -139,7 +141,7 @@ size_t topk_merge_workspace(int64_t rows, int k) {
 
 cudaError_t launch_topk_merge(int64_t rows, int n_parts, int k, const float* cand_scores, const int32_t* cand_ids,
                               int64_t entry0, int64_t n_entries, int32_t* sel_global, int32_t* sel_local,
-                              void* ws, int m, int W, cudaStream_t s) {
+                              int32_t* n_local, void* ws, int m, int W, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
     const int n_cand = n_parts * k;
     if (!topk_merge_supported(n_cand, k)) return cudaErrorInvalidValue;
@@ -156,7 +158,7 @@ cudaError_t launch_topk_merge(int64_t rows, int n_parts, int k, const float* can
     e = launch_topk(row_scores, n_cand, n_cand, pos, m, W, k, rows, sel_pos, s);
     if (e != cudaSuccess) return e;
     map_selection_kernel<<<unsigned(rows), kMapThreads, 0, s>>>(rows, n_parts, k, sel_pos, cand_ids, entry0,
-                                                                n_entries, sel_global, sel_local);
+                                                                n_entries, sel_global, sel_local, n_local);
     return cudaGetLastError();
 }
 

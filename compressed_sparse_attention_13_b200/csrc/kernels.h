@@ -30,6 +30,8 @@ struct AttnArgs {
     int partial_out;          // write (m, l, O) partials even with one split; no sink applied
     int64_t kv_base;          // global index of entry 0 of kv (a shard); dense rows attend to
                               // entries j with kv_base + j < n_elig(t)
+    const int32_t* n_sel;     // [rows] or null: row r's selection is compacted, only its first
+                              // n_sel[r] slots can hold ids (the slots after them are -1)
 };
 
 cudaError_t launch_compress(int in_fmt, int out_fmt, const void* x, const void* z,
@@ -97,6 +99,6 @@ bool topk_merge_supported(int n_cand, int k);
 size_t topk_merge_workspace(int64_t rows, int k);
 cudaError_t launch_topk_merge(int64_t rows, int n_parts, int k, const float* cand_scores, const int32_t* cand_ids,
                               int64_t entry0, int64_t n_entries, int32_t* sel_global, int32_t* sel_local,
-                              void* ws, int m, int W, cudaStream_t s);
+                              int32_t* n_local, void* ws, int m, int W, cudaStream_t s);
 
 }  // namespace csa
