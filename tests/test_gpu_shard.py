@@ -18,6 +18,7 @@ import torch
 
 import compressed_sparse_attention_13_b200 as K
 import oracle
+import synth
 from compressed_sparse_attention_13_b200 import shard as SH
 from helpers import (assert_attention_close, attention_bound_stored, both_stored, check_selection, down,
                      orc_quantize, sink_dominant, up)
@@ -142,3 +143,54 @@ def test_attn_merge_of_one_part_is_the_normalised_partial():
     ref_o = oracle.attention(*args, None, [65536], H, m, W, w.scale)[0]
     bound = attention_bound_stored(*args, None, [65536], H, m, W, w.scale)[0]
     assert_attention_close(got[0], ref_o, bound, "one-part merge")
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_fp32_sharded_decode_matches_oracle_to_1e5(world):
+    """The fp32 formats (CUDA-core indexer and attention, fp32 entries) through
+    the sharded CSA and HCA paths: the merged outputs match the oracle's
+    unsharded attention within 1e-5, which pins the partial (M, L, O) and the
+    LSE merge arithmetic tightly; the selection is valid against the oracle's
+    scores."""
+    from helpers import assert_close_f32
+    B, H, d, HI, dI, m, W, k = 2, 8, 64, 4, 32, 4, 64, 16
+    rng_seed = 61
+    nb = 1024
+    st = lambda a: oracle.Stored(oracle.F32, np.ascontiguousarray(a, np.float32).reshape(-1, a.shape[-1]))
+    q_h = synth.tensor_np(rng_seed, "f32s/q", (B, H, d))
+    qI_h = synth.tensor_np(rng_seed, "f32s/qI", (B, HI, dI))
+    w_h = synth.tensor_np(rng_seed, "f32s/w", (B, HI), std=0.1)
+    kv_h = synth.tensor_np(rng_seed, "f32s/kv", (B, nb, d))
+    kI_h = synth.tensor_np(rng_seed, "f32s/kI", (B, nb, dI))
+    win_h = synth.tensor_np(rng_seed, "f32s/win", (B, W, d))
+    sinks = synth.tensor_np(rng_seed, "f32s/sinks", (H,))
+    q_pos = np.array([m * nb + W, m * 300 + W + 3], np.int64)
+    raw_pos0 = q_pos - W + 1
+    p = K.params(m, W, k, H, d, HI, dI, 1 / 8, K.F32, K.F32, K.F32)
+    kv_d = K.Stored(K.F32, up(kv_h.reshape(-1, d)))
+    kI_d = K.Stored(K.F32, up(kI_h.reshape(-1, dI)))
+    shards = SH.make_shards(kv_d, kI_d, B, nb, world)
+    out = torch.empty(B, H, d, dtype=torch.float32, device="cuda")
+    sel = torch.empty(B, k, dtype=torch.int32, device="cuda")
+    SH.emulate_csa_layer(p, B, up(q_h), K.Stored(K.F32, up(qI_h.reshape(-1, dI))), up(w_h), shards, up(win_h), W,
+                         up(raw_pos0), up(q_pos), up(sinks), out, idx_out=sel)
+    torch.cuda.synchronize()
+    got, got_sel = down(out), down(sel)
+    for b in range(B):
+        t = int(q_pos[b])
+        scores = oracle.indexer(st(qI_h[b]), w_h[b][None], st(kI_h[b]), [t], HI, m, W)[0]
+        check_selection(got_sel[b], scores, min(oracle.n_elig(t, m, W), nb), k, what=f"fp32 seq {b}")
+        ref = oracle.attention(st(q_h[b]), st(kv_h[b]), got_sel[b][None], st(win_h[b]), t - W + 1, sinks, [t], H, m,
+                               W, 1 / 8)[0]
+        assert_close_f32(got[b], ref, 1e-5, f"fp32 sharded csa seq {b}")
+    # HCA at m' = 16 over the same entries
+    ph = K.params(16, W, 1, H, d, 1, 32, 1 / 8, K.F32, K.F32, K.F32)
+    qh_pos = np.array([16 * nb + W, 16 * 200 + W + 5], np.int64)
+    hsh = SH.make_shards(kv_d, None, B, nb, world)
+    SH.emulate_hca_layer(ph, B, up(q_h), hsh, up(win_h), W, up(qh_pos - W + 1), up(qh_pos), up(sinks), out)
+    torch.cuda.synchronize()
+    got = down(out)
+    for b in range(B):
+        t = int(qh_pos[b])
+        ref = oracle.attention(st(q_h[b]), st(kv_h[b]), None, st(win_h[b]), t - W + 1, sinks, [t], H, 16, W, 1 / 8)[0]
+        assert_close_f32(got[b], ref, 1e-5, f"fp32 sharded hca seq {b}")
