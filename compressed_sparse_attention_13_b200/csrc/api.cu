@@ -541,7 +541,7 @@ int csa_shard_attend(const csa_params* p, int32_t batch, const void* q, int32_t 
     if (st) return st;
     if (p->top_k <= 0 || batch < 0 || n_parts <= 0 || n_entries < 0 || entry0 < 0) return CSA_ERR_ARG;
     if (batch == 0) return CSA_OK;
-    if (!topk_merge_supported(n_parts * p->top_k, p->top_k)) return CSA_ERR_UNSUPPORTED;
+    if (n_parts > 64 || !topk_merge_supported(n_parts * p->top_k, p->top_k)) return CSA_ERR_UNSUPPORTED;
     if (!cand_scores || !cand_ids || !part_ml || !workspace) return CSA_ERR_ARG;
     st = check_attn_ptrs(q, kv, kv_scales, p->kv_fmt, raw, n_raw, raw_pos0, q_pos, part_o, n_entries > 0);
     if (st) return st;

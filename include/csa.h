@@ -382,8 +382,8 @@ int csa_shard_select(const csa_params* p, int32_t batch, const void* qI, const v
 /* csa_shard_attend -- the global top-k of the gathered candidates and this
  * rank's partial of the sparse attention.
  *   cand_scores, cand_ids: [n_parts][batch][k] (every rank's csa_shard_select
- *   output, rank-major); n_parts * k <= 16384 and k <= 4096, else
- *   CSA_ERR_UNSUPPORTED.  kv: this rank's entries [batch][n_entries][d] in
+ *   output, rank-major); n_parts <= 64, n_parts * k <= 16384 and k <= 4096,
+ *   else CSA_ERR_UNSUPPORTED.  kv: this rank's entries [batch][n_entries][d] in
  *   p->kv_fmt; raw / n_raw / raw_pos0: the window as for csa_decode on the
  *   rank that attends to it, n_raw = 0 (raw may be NULL) elsewhere.
  *   part_o float [batch][H][d], part_ml float [batch][H][2]: the partial.

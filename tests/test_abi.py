@@ -233,3 +233,14 @@ def test_sharded_decode_host_errors():
     assert lib.attn_merge(P, 1, 65, fake, fake, None, fake, None) == -3
     odd = C.c_void_p(0x1004)
     assert lib.attn_merge(P, 1, 2, odd, fake, None, fake, None) == -2
+
+
+def test_shard_attend_refuses_more_than_64_parts():
+    lib = K.lib()
+    p = K.params(4, 128, 16, 64, 512, 64, 128, 0.044)
+    fake = C.c_void_p(0x1000)
+    # 2^20 + 1 parts of 4096 would wrap a 32-bit product: refused before it is formed
+    big = K.params(4, 128, 4096, 64, 512, 64, 128, 0.044)
+    for P, n in ((p, 65), (big, (1 << 20) + 1)):
+        assert lib.csa_shard_attend(C.byref(P), 1, fake, n, fake, fake, fake, fake, 1024, 0, None, 0, fake, fake,
+                                    fake, fake, None, fake, 1 << 30, None) == -3
