@@ -499,17 +499,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) ok = mbar_wait(&S.s_full[kb], uint32_t((tile >> 1) & 1));
             if (ok) tc_fence_after();
             const uint32_t srow = tS + 64 * kb + (uint32_t(sub * 32) << 16);
-            // pass 1: max of the scaled, masked logits (two 32-item halves)
+            // lanes 0-15 hold items 0..31 of head h, lanes 16-31 items 32..63
+            const bool upper = lane >= 16;
+            const unsigned vm = upper ? vm1 : vm0;
+            float x[32];
+            if (ok) tmem_ld16x2_32(srow, x);
+            // the max of the scaled, masked logits over both halves
             float mx = -INFINITY;
-#pragma unroll 1
-            for (int hf = 0; hf < 2; ++hf) {  // rolled: one 32-column half live at a time
-                float x[32];
-                if (ok) tmem_ld32(srow + 32 * hf, x);
-                const unsigned vm = hf ? vm1 : vm0;
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (ok && ((vm >> i) & 1u)) mx = fmaxf(mx, x[i] * sl2);
-            }
+            for (int i = 0; i < 32; ++i)
+                if (ok && ((vm >> i) & 1u)) mx = fmaxf(mx, x[i] * sl2);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
             float al = 1.f;
             if (mx > m_run + kRescaleThreshold || (m_run == -INFINITY && mx != -INFINITY)) {
                 al = m_run == -INFINITY ? 0.f : ex2(m_run - mx);
@@ -518,31 +518,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             // P[kb] was read by P.V two tiles back: that one must be done (its
             // completion also releases the tile buffer, hence kv_empty)
             if (ok && tile >= 2) ok = mbar_wait(&S.kv_empty[kb], uint32_t(((tile >> 1) - 1) & 1));
-            // pass 2: P = exp2(x - m) as bf16 rows of the K-major B tile, and the sum
+            // P = exp2(x - m) as bf16 rows of the K-major B tile (each lane its
+            // 32 items: 16-byte chunks 0-3 or 4-7 of row h), and the sum
             float sum = 0.f;
-#pragma unroll 1
-            for (int hf = 0; hf < 2; ++hf) {
-                float x[32];
-                if (ok) tmem_ld32(srow + 32 * hf, x);
-                const unsigned vm = hf ? vm1 : vm0;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    x[i] = (ok && ((vm >> i) & 1u)) ? ex2(x[i] * sl2 - m_run) : 0.f;
-                    sum += x[i];
+            for (int i = 0; i < 32; ++i) {
+                x[i] = (ok && ((vm >> i) & 1u)) ? ex2(x[i] * sl2 - m_run) : 0.f;
+                sum += x[i];
+            }
+            sum += __shfl_xor_sync(0xffffffffu, sum, 16);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const __nv_bfloat162 hh = __floats2bfloat162_rn(x[8 * ch + 2 * k], x[8 * ch + 2 * k + 1]);
+                    w4[k] = *reinterpret_cast<const uint32_t*>(&hh);
                 }
-                if (head_lane) {
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t w4[4];
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const __nv_bfloat162 hh = __floats2bfloat162_rn(x[8 * ch + 2 * k], x[8 * ch + 2 * k + 1]);
-                            w4[k] = *reinterpret_cast<const uint32_t*>(&hh);
-                        }
-                        *reinterpret_cast<uint4*>(S.p[kb] + sw128_offset(h, 4 * hf + ch)) =
-                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    }
-                }
+                *reinterpret_cast<uint4*>(S.p[kb] + sw128_offset(h, 4 * int(upper) + ch)) =
+                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
             l_run = l_run * al + sum;
             if (head_lane) {
