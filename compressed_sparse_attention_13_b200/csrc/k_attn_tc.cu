@@ -225,42 +225,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cp_async_wait_all();
             } else if (kFp8 && tile0 + lt < kv_tiles) {
                 const uint8_t* raw = S.kv[kb][kRawBlk];  // [64 items][512 E4M3] over blocks 4..7
-                // dims 0..255 -> lower half (the rows sit in the upper half)
+                // every code and scale of this thread's units is read first (16
+                // independent shared-memory loads in flight), then converted:
+                // dims 0..255 to the lower half (the rows sit in the upper half)
+                uint2 w[4][kUnits];
+                float sc[4][kUnits];
+#pragma unroll
+                for (int qt = 0; qt < 4; ++qt)
+#pragma unroll
+                    for (int u = 0; u < kUnits; ++u) {
+                        const int item = e0 + 16 * u;
+                        const bool v = S.valid[kb][item] != 0;
+                        w[qt][u] = v ? *reinterpret_cast<const uint2*>(raw + kD * item + 128 * qt + 8 * c)
+                                     : make_uint2(0, 0);
+                        sc[qt][u] = v ? S.kvs[kb][item][(128 * qt + 8 * c) >> 6] : 0.f;
+                    }
 #pragma unroll
                 for (int qt = 0; qt < 2; ++qt)
 #pragma unroll
                     for (int u = 0; u < kUnits; ++u) {
                         const int item = e0 + 16 * u;
-                        uint4 o = make_uint4(0, 0, 0, 0);
-                        if (S.valid[kb][item])
-                            o = dequant8(*reinterpret_cast<const uint2*>(raw + kD * item + 128 * qt + 8 * c),
-                                         S.kvs[kb][item][(128 * qt + 8 * c) >> 6]);
-                        *reinterpret_cast<uint4*>(S.kv[kb][2 * qt + (c >> 3)] + sw128_offset(item, c & 7)) = o;
+                        *reinterpret_cast<uint4*>(S.kv[kb][2 * qt + (c >> 3)] + sw128_offset(item, c & 7)) =
+                            dequant8(w[qt][u], sc[qt][u]);
                     }
                 // the product over dims 0..255 may start while the upper half converts
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.kv_half[kb]);
-                // dims 256..511: read everything first, then overwrite the upper half
-                uint2 w[2][kUnits];
-                float sc[2][kUnits];
-#pragma unroll
-                for (int qt = 0; qt < 2; ++qt)
-#pragma unroll
-                    for (int u = 0; u < kUnits; ++u) {
-                        const int item = e0 + 16 * u;
-                        const bool v = S.valid[kb][item] != 0;
-                        w[qt][u] = v ? *reinterpret_cast<const uint2*>(raw + kD * item + 128 * (qt + 2) + 8 * c)
-                                     : make_uint2(0, 0);
-                        sc[qt][u] = v ? S.kvs[kb][item][(128 * (qt + 2) + 8 * c) >> 6] : 0.f;
-                    }
+                // dims 256..511 overwrite the raw rows once every converter has read them
                 named_bar(2, kConvThreads);
 #pragma unroll
-                for (int qt = 0; qt < 2; ++qt)
+                for (int qt = 2; qt < 4; ++qt)
 #pragma unroll
                     for (int u = 0; u < kUnits; ++u) {
                         const int item = e0 + 16 * u;
-                        *reinterpret_cast<uint4*>(S.kv[kb][2 * (qt + 2) + (c >> 3)] + sw128_offset(item, c & 7)) =
+                        *reinterpret_cast<uint4*>(S.kv[kb][2 * qt + (c >> 3)] + sw128_offset(item, c & 7)) =
                             dequant8(w[qt][u], sc[qt][u]);
                     }
             } else {
