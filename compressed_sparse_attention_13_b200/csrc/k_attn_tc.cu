@@ -681,14 +681,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int lo = r * n4 / ns, hi = (r + 1) * n4 / ns;
         const float4* part = reinterpret_cast<const float4*>(&S.kv[0][0][0]);
         __nv_bfloat16* out = (__nv_bfloat16*)a.out + row * int64_t(kH) * kD;
+        // the splits' partials of a position are all requested before any is
+        // used (at most 8 remote loads in flight per thread), then summed in
+        // split order
+        const float4* rp[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) rp[q] = q < ns ? cl.map_shared_rank(part, q) : part;
         for (int i = lo + threadIdx.x; i < hi; i += kThreads) {
             const int hh = (4 * i) / kD;
+            float4 v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (q < ns) v[q] = rp[q][i];
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int q = 0; q < ns; ++q) {
-                const float4 v = cl.map_shared_rank(part, q)[i];
-                const float wq = S.cw[q][hh];
-                acc.x += wq * v.x; acc.y += wq * v.y; acc.z += wq * v.z; acc.w += wq * v.w;
-            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (q < ns) {
+                    const float wq = S.cw[q][hh];
+                    acc.x += wq * v[q].x; acc.y += wq * v[q].y; acc.z += wq * v[q].z; acc.w += wq * v[q].w;
+                }
             const float inv = S.cinv[hh];
             const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
             const __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
