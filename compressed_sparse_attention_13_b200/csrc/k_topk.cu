@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_smem_kernel(
 constexpr int kWarpRowMax = 2048;
 constexpr int kWarpRowThreads = 128;  // 4 rows per CTA
 
-__global__ void __launch_bounds__(kWarpRowThreads) topk_warp_kernel(
+__global__ void __launch_bounds__(kWarpRowThreads, 6) topk_warp_kernel(
     const float* __restrict__ scores, int64_t ld, int64_t max_blocks, const int64_t* __restrict__ q_pos, int m,
     int W, int k, int64_t rows, int32_t* __restrict__ idx) {
     constexpr int kPer = kWarpRowMax / 32;
