@@ -57,7 +57,7 @@ typedef enum csa_status {
     CSA_OK = 0,
     CSA_ERR_ARG = -1,         /* null pointer, non-positive size, inconsistent parameters */
     CSA_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned */
-    CSA_ERR_UNSUPPORTED = -3, /* a shape / format combination this build does not implement */
+    CSA_ERR_UNSUPPORTED = -3, /* a shape / format combination this library does not implement */
     CSA_ERR_WORKSPACE = -4,   /* workspace smaller than csa_workspace_size() */
     CSA_ERR_CUDA = -5         /* a kernel launch failed (the CUDA error is not cleared) */
 } csa_status;
