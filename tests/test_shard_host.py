@@ -146,19 +146,26 @@ def test_shard_bounds_cover_the_entries():
         assert all(b[r][1] % 128 == 0 for r in range(last))   # all but the last non-empty shard
 
 
-def test_sharded_csa_and_hca_two_gloo_ranks_match_the_oracle():
-    world = 2
-    port = 29700 + os.getpid() % 200
+@pytest.mark.parametrize("world", [2, 4])
+def test_sharded_csa_and_hca_gloo_ranks_match_the_oracle(world):
+    """Two ranks; and four, where the last HCA shard (the window rank) holds
+    no entries: 300 entries in shards of 128, 128, 44 and 0."""
+    port = 29700 + (os.getpid() * 7 + world) % 200
     with mp.Manager() as m:
         res = m.dict()
         mp.start_processes(_rank, args=(world, port, res), nprocs=world, start_method="spawn")
         res = dict(res)
-    assert res[0][3] == (0, 512) and res[1][3] == (512, N_CSA - 512)
+    assert [res[r][3] for r in range(world)] == [SH.shard_bounds(N_CSA, world, r) for r in range(world)]
+    if world == 2:
+        assert res[0][3] == (0, 512) and res[1][3] == (512, N_CSA - 512)
+    if world == 4:
+        assert [res[r][4] for r in range(world)] == [(0, 128), (128, 128), (256, 44), (300, 0)]
     d = _data()
     q_pos = np.array([M_CSA * N_CSA + W, 2500], np.int64)
     for r in range(world):                    # every rank merged the same result
         np.testing.assert_array_equal(res[r][0], res[0][0])
         np.testing.assert_array_equal(res[r][1], res[0][1])
+        np.testing.assert_array_equal(res[r][2], res[0][2])
     for b in range(B):
         t = int(q_pos[b])
         s = oracle.indexer(_st(d["qI"][b]), d["w"][b][None], _st(d["kI"][b]), [t], HI, M_CSA, W)[0]
@@ -172,4 +179,4 @@ def test_sharded_csa_and_hca_two_gloo_ranks_match_the_oracle():
         t = int(qh_pos[b])
         ref = oracle.attention(_st(d["q"][b]), _st(d["kv_h"][b]), None, _st(d["win"][b]), t - W + 1, d["sinks"],
                                [t], H, M_HCA, W, 1 / np.sqrt(D))[0]
-        np.testing.assert_allclose(res[1][2][b], ref, rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(res[0][2][b], ref, rtol=1e-9, atol=1e-12)
