@@ -11,7 +11,8 @@ one GPU: the same C-ABI calls per rank and the same exchanged tensors
     bound).
   * HCA: the merged output matches the oracle's dense attention.
 Cases: 1, 3 and 4 ranks; shards that end past a sequence's eligible entries
-(a rank with nothing visible); uneven last shards; sink-dominant logits."""
+(a rank with nothing visible); uneven last shards; a window rank that holds
+no entries; sink-dominant logits."""
 import numpy as np
 import pytest
 import torch
@@ -48,6 +49,7 @@ def _bf16_orc(bits):
     (1, 16384, [16384, 9000]),
     (3, 32768, [32768, 12000]),       # ranks 1-2 see few or no eligible entries of sequence 1
     (4, 32768 + 4 * 128, [33280, 20001]),  # uneven last shard
+    (4, 1200, [1200, 700]),           # 300 entries: shards of 128, 128, 44 and none (the window rank)
 ])
 def test_csa_sharded_decode_matches_unsharded_selection_and_oracle(world, n_ctx, q_pos):
     w = WORKLOADS["csa_decode_128k_b32"].with_(batch=2, n_ctx=n_ctx, seed=23)
