@@ -1,6 +1,7 @@
 """The multi-GPU bench path (independent replicas, one per rank) on CPU:
 world-size-2 gloo ranks check the max-over-ranks timing and the whole-job
-throughput, and that the reference arm runs on rank 0 only."""
+throughput, and that the reference arm runs on rank 0 only and prints one
+contract line."""
 import json
 import os
 import subprocess
@@ -57,3 +58,25 @@ def test_reference_arm_runs_on_rank_zero_only():
                        timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_reference_arm_prints_one_contract_line():
+    """The reference arm alone (one process): one JSON line with the same
+    metric, unit and workload as the library's arm, the oracle's timing as
+    its value, a cpu_baseline describing that run and an e2e with no host
+    copies."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 3
+    assert d["unit"] == "tok/s" and d["higher_is_better"] is True and d["vs_baseline"] is None
+    assert d["config"]["workload"] == "csa_decode_128k_b32" and d["config"]["batch"] == 32
+    assert d["value"] > 0 and d["ms_per_step"] > 0
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
