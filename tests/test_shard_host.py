@@ -180,3 +180,43 @@ def test_sharded_csa_and_hca_gloo_ranks_match_the_oracle(world):
         ref = oracle.attention(_st(d["q"][b]), _st(d["kv_h"][b]), None, _st(d["win"][b]), t - W + 1, d["sinks"],
                                [t], H, M_HCA, W, 1 / np.sqrt(D))[0]
         np.testing.assert_allclose(res[0][2][b], ref, rtol=1e-9, atol=1e-12)
+
+
+def _merge_by_position(cand_s, cand_i, k):
+    """The selection rule of the library's candidate merge: the rank-major
+    candidates of a row side by side, the k best positions by score with
+    ties to the lower position, empty slots dropped, ids ascending."""
+    order = np.lexsort((np.arange(cand_s.size), -cand_s.astype(np.float64)))[:k]
+    ids = cand_i[order]
+    return np.sort(ids[ids >= 0])
+
+
+def test_merge_of_local_topk_by_position_equals_the_global_topk():
+    """With heavy ties, random shard counts and eligible counts: the merge of
+    the shards' local top-k (each at the shifted position t - entry0 * m)
+    selects exactly the oracle's top-k of the whole row, because ranks hold
+    increasing id ranges and list their candidates ascending."""
+    rng = np.random.default_rng(11)
+    m, W = 4, 8
+    for _ in range(300):
+        n = int(rng.integers(1, 400))
+        k = int(rng.integers(1, 48))
+        world = int(rng.integers(1, 7))
+        scores = rng.integers(-3, 4, n).astype(np.float32)
+        t = W + m * int(rng.integers(0, n + 3)) + int(rng.integers(0, m))
+        cs, ci = [], []
+        for r in range(world):
+            e0, nr = SH.shard_bounds(n, world, r, align=8)
+            s_loc = np.full(k, -np.inf, np.float32)
+            i_loc = np.full(k, -1, np.int32)
+            if nr:
+                t_loc = t - e0 * m
+                sel = oracle.topk(scores[e0:e0 + nr][None], [t_loc], k, m, W)[0]
+                ok = sel >= 0
+                s_loc[ok] = scores[e0 + sel[ok]]
+                i_loc[ok] = sel[ok] + e0
+            cs.append(s_loc)
+            ci.append(i_loc)
+        got = _merge_by_position(np.concatenate(cs), np.concatenate(ci), k)
+        want = oracle.topk(scores[None], [t], k, m, W)[0]
+        np.testing.assert_array_equal(got, want[want >= 0], err_msg=f"n={n} k={k} world={world} t={t}")
