@@ -37,12 +37,15 @@ def shard_bounds(n_total: int, world: int, rank: int, align: int = 128):
 
 
 def nccl_gather(t):
-    """All-gather over the default process group, rank-major."""
+    """All-gather over the default process group, rank-major
+    [world, *t.shape]: one collective into one buffer (flattened, so every
+    backend splits it by rank the same way), with no per-rank copies."""
     import torch
     import torch.distributed as dist
-    parts = [torch.empty_like(t) for _ in range(dist.get_world_size())]
-    dist.all_gather(parts, t.contiguous())
-    return torch.stack(parts)
+    world = dist.get_world_size()
+    out = torch.empty(world * t.numel(), dtype=t.dtype, device=t.device)
+    dist.all_gather_into_tensor(out, t.contiguous().reshape(-1))
+    return out.view((world,) + tuple(t.shape))
 
 
 @dataclass
