@@ -220,3 +220,38 @@ def test_merge_of_local_topk_by_position_equals_the_global_topk():
         got = _merge_by_position(np.concatenate(cs), np.concatenate(ci), k)
         want = oracle.topk(scores[None], [t], k, m, W)[0]
         np.testing.assert_array_equal(got, want[want >= 0], err_msg=f"n={n} k={k} world={world} t={t}")
+
+
+def test_make_shards_slices_every_sequence_and_its_scales():
+    """make_shards gives rank r the rows [entry0, entry0 + n) of every
+    sequence of a stored [batch][n_total] cache, codes and scales alike, as
+    contiguous [batch * n] tensors; the window goes to the last rank unless
+    another is named (host logic; CPU tensors)."""
+    import compressed_sparse_attention_13_b200 as K
+    batch, n_total, d, dI, world = 3, 700, 128, 64, 4
+    g = torch.Generator().manual_seed(3)
+    kv = K.empty_stored(K.FP8_S64, batch * n_total, d, device="cpu")
+    kv.data.copy_(torch.randint(0, 256, kv.data.shape, generator=g, dtype=torch.uint8))
+    kv.scales.copy_(torch.rand(kv.scales.shape, generator=g))
+    kI = K.empty_stored(K.MXFP4, batch * n_total, dI, device="cpu")
+    kI.data.copy_(torch.randint(0, 256, kI.data.shape, generator=g, dtype=torch.uint8))
+    kI.scales.copy_(torch.randint(0, 256, kI.scales.shape, generator=g, dtype=torch.uint8))
+    for window_rank in (None, 1):
+        shards = SH.make_shards(kv, kI, batch, n_total, world, window_rank)
+        assert [s.window for s in shards] == [r == (world - 1 if window_rank is None else 1) for r in range(world)]
+        for r, sh in enumerate(shards):
+            assert (sh.entry0, sh.n) == SH.shard_bounds(n_total, world, r)
+            for st, full in ((sh.kv, kv), (sh.kI, kI)):
+                assert st.fmt == full.fmt
+                for part, whole in ((st.data, full.data), (st.scales, full.scales)):
+                    assert part.is_contiguous() and part.shape == (batch * sh.n, whole.shape[1])
+                    want = whole.reshape(batch, n_total, -1)[:, sh.entry0:sh.entry0 + sh.n].reshape(-1, whole.shape[1])
+                    assert torch.equal(part, want)
+    assert SH.make_shards(kv, None, batch, n_total, 2)[0].kI is None
+
+
+def test_exchange_bytes():
+    """A CSA step exchanges k (score, id) pairs and the partial (O and (M, L)
+    per head, fp32); an HCA step the partial alone."""
+    assert SH.exchange_bytes(1, 1024, 64, 512, csa=True) == 1024 * 8 + 64 * 514 * 4
+    assert SH.exchange_bytes(2, 512, 8, 64, csa=False) == 2 * 8 * 66 * 4
