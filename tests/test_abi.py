@@ -16,7 +16,8 @@ def _declared():
     for fn in os.listdir(os.path.join(ROOT, "include")):
         if not fn.endswith(".h"):
             continue
-        src = open(os.path.join(ROOT, "include", fn)).read()
+        with open(os.path.join(ROOT, "include", fn)) as f:
+            src = f.read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
         for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", src, re.M):
             if m.group(1) not in ("if", "sizeof", "defined"):

@@ -36,7 +36,7 @@ def _rank(rank, world, port, times, out):
 def test_max_over_ranks_and_job_throughput_two_gloo_ranks():
     world, times = 2, [17.5, 23.25]
     port = 29500 + os.getpid() % 1000
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:   # no fork of a threaded process
         out = m.dict()
         mp.start_processes(_rank, args=(world, port, times, out), nprocs=world, start_method="spawn")
         res = dict(out)

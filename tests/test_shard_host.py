@@ -151,7 +151,7 @@ def test_sharded_csa_and_hca_gloo_ranks_match_the_oracle(world):
     """Two ranks; and four, where the last HCA shard (the window rank) holds
     no entries: 300 entries in shards of 128, 128, 44 and 0."""
     port = 29700 + (os.getpid() * 7 + world) % 200
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:   # no fork of a threaded process
         res = m.dict()
         mp.start_processes(_rank, args=(world, port, res), nprocs=world, start_method="spawn")
         res = dict(res)
