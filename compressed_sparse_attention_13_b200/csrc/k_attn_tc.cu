@@ -407,16 +407,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // loop as a whole is bounded by kWaitNs without progress.
             // QK of a tile runs in two halves over the dims: 0..255 once the
             // converters have written them, 256..511 once the whole tile is in
-            // With at most three tiles the third one's copy waits for P.V of the
-            // first (two tile buffers), so P.V(t) goes to the tensor pipe
-            // before QK(t+1); longer rows keep QK one tile ahead so that it
-            // overlaps the softmax.
-            const int lead = n_tiles <= 3 ? 0 : 1;
             int qk_t = 0, pv_t = 0, qk_half = 0;
             uint64_t t_last = global_ns();
             while (ok && pv_t < n_tiles) {
                 bool progressed = false;
-                if (qk_t < n_tiles && qk_t <= pv_t + lead) {
+                if (qk_t < n_tiles && qk_t <= pv_t + 1) {
                     const int kb = qk_t & 1;
                     const uint32_t par = uint32_t((qk_t >> 1) & 1);
                     if (mbar_test_wait(qk_half ? &S.kv_full[kb] : &S.kv_half[kb], par)) {
