@@ -17,8 +17,9 @@
 //   * HCA: the same pooling at m' = 128 tokens per entry and dense attention
 //     over all pooled entries plus the same window.  (Release note, section
 //     重度壓縮注意力 (HCA); wiki summary, HCA bullet.)
-//   * Sliding-window branch and an attention sink.  (Wiki summary, 架构创新,
-//     "两者交替配置，配合滑动窗口注意力分支和 Attention Sink".)
+//   * Sliding-window branch and an attention sink.  (Wiki summary, section
+//     架构创新: the two kinds of layer alternate and are joined by a
+//     sliding-window branch and an attention sink.)
 //   * FP8 storage of KV entries and FP4 for the indexer QK path.  (Release
 //     note, section 架構實現; wiki summary, section 基础设施, FP4 QAT bullet.)
 //
